@@ -1,0 +1,306 @@
+// Epilogues for the tcgen05 GEMM engine.  Each runs on the 128 epilogue
+// threads; thread i owns accumulator row `row` (TMEM lane) of the current
+// 128 x BN tile and reads its BN fp32 columns from TMEM in chunks of 32.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace twell {
+
+// Row-slot protocol for the hybrid dense backup ("Sparser, Faster, Lighter
+// Transformer Language Models", §3-6 and §4-3: rows over capacity go to a dense
+// backup of bounded size).  row_slot[m] is -1 (free) until the first tile of
+// row m overflows; that thread swaps in kSlotPending, takes the next slot from
+// the n_over counter and publishes it.  Other tiles of the same row wait
+// (bounded) for the publication.  Slots past R_cap publish kSlotNoCapacity.
+constexpr int kSlotFree = -1;
+constexpr int kSlotNoCapacity = -2;
+constexpr int kSlotPending = -3;
+
+__device__ __forceinline__ int acquire_row_slot(int* row_slot, int* slot_row, int r_cap, int row, int* ctrl,
+                                                bool& fresh) {
+  fresh = false;
+  int s = atomicCAS(row_slot + row, kSlotFree, kSlotPending);
+  if (s == kSlotFree) {
+    const int ns = atomicAdd(ctrl + kCtrlNOver, 1);
+    if (ns < r_cap) {
+      slot_row[ns] = row;
+      s = ns;
+      fresh = true;
+    } else {
+      s = kSlotNoCapacity;
+      set_flag(ctrl, kFlagNoCapacity);
+    }
+    atomicExch(row_slot + row, s);
+    return s;
+  }
+  if (s != kSlotPending) return s;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    s = atomicAdd(row_slot + row, 0);
+    if (s != kSlotPending) return s;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      set_flag(ctrl, kFlagWaitTimeout);
+      return kSlotNoCapacity;
+    }
+  }
+}
+
+__device__ __forceinline__ float relu_f(float z) { return z > 0.f ? z : 0.f; }
+
+// ---------------------------------------------------------------------------
+// Gate epilogue: ReLU + TwELL packing + overflow routing ("Sparser, Faster,
+// Lighter Transformer Language Models", §3-4 steps 3-5 and §3-6).
+// The tile width T equals BN, so a (row, tile) record is produced entirely by
+// one thread from its own TMEM lane: no cross-CTA or cross-thread step.
+struct EpiGateTwell {
+  struct Params {
+    uint16_t* counts;      // [M][N/T]
+    uint8_t* idx;          // [M][N/T][C]
+    float* vals;           // [M][N/T][C]
+    float* dense_rows;     // [R_cap][N]
+    int* row_slot;         // [M]
+    int* slot_row;         // [R_cap]
+    const uint16_t* x;     // [M][K] gate input, copied to x_over for slotted rows
+    uint16_t* x_over;      // [R_cap][K]
+    int N, K, C, r_cap;
+  };
+
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb,
+                                             int lane, int* ctrl) {
+    const bool valid = row < m_rows;
+    const int NT = p.N / BN;
+    const int64_t rec = static_cast<int64_t>(row) * NT + nb;
+    uint8_t* idx_rec = p.idx + rec * p.C;
+    float* val_rec = p.vals + rec * p.C;
+    int cnt = 0;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32(taddr + c * 32, r);
+      tmem_wait_ld();
+      if (valid) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float z = __uint_as_float(r[j]);
+          if (z > 0.f) {
+            if (cnt < p.C) {
+              idx_rec[cnt] = static_cast<uint8_t>(c * 32 + j);
+              val_rec[cnt] = z;
+            }
+            ++cnt;
+          }
+        }
+      }
+    }
+    if (valid) p.counts[rec] = static_cast<uint16_t>(cnt);
+    const bool ov = valid && cnt > p.C;
+    if (__any_sync(0xffffffffu, ov)) {
+      int slot = -1;
+      bool fresh = false;
+      if (ov) slot = acquire_row_slot(p.row_slot, p.slot_row, p.r_cap, row, ctrl, fresh);
+      // The lane that opened a slot brings its x row along (whole warp copies).
+      uint32_t fresh_mask = __ballot_sync(0xffffffffu, fresh);
+      while (fresh_mask) {
+        const int src = __ffs(fresh_mask) - 1;
+        fresh_mask &= fresh_mask - 1;
+        const int r = __shfl_sync(0xffffffffu, row, src);
+        const int sl = __shfl_sync(0xffffffffu, slot, src);
+        const uint4* xs = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.K);
+        uint4* xd = reinterpret_cast<uint4*>(p.x_over + static_cast<int64_t>(sl) * p.K);
+        for (int v = lane; v < p.K / 8; v += 32) xd[v] = xs[v];
+      }
+      float* dst = slot >= 0 ? p.dense_rows + static_cast<int64_t>(slot) * p.N + nb * BN : nullptr;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32(taddr + c * 32, r);
+        tmem_wait_ld();
+        if (dst) {
+          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            d4[v] = make_float4(relu_f(__uint_as_float(r[4 * v + 0])), relu_f(__uint_as_float(r[4 * v + 1])),
+                                relu_f(__uint_as_float(r[4 * v + 2])), relu_f(__uint_as_float(r[4 * v + 3])));
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Dense FFN first stage: accumulator 0 = x W_g tile, accumulator 1 = x W_u
+// tile (same columns).  Writes h = h_u * ReLU(h_g) as bf16 ("Sparser, Faster,
+// Lighter Transformer Language Models", §1-1).
+struct EpiGatedProduct {
+  struct Params {
+    uint16_t* h;  // [M][N] bf16
+    int N;
+  };
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
+                                             int*) {
+    const bool valid = row < m_rows;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t g[32], u[32];
+      tmem_ld_32x32(taddr + c * 32, g);
+      tmem_ld_32x32(taddr + BN + c * 32, u);
+      tmem_wait_ld();
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.h + static_cast<int64_t>(row) * p.N + nb * BN + c * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          float h[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) h[e] = __uint_as_float(u[8 * v + e]) * relu_f(__uint_as_float(g[8 * v + e]));
+          uint4 o;
+          o.x = pack_bf16x2(h[0], h[1]);
+          o.y = pack_bf16x2(h[2], h[3]);
+          o.z = pack_bf16x2(h[4], h[5]);
+          o.w = pack_bf16x2(h[6], h[7]);
+          dst[v] = o;
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Plain fp32 store of the accumulator: y[row][col] = acc, col < ncols.
+struct EpiStoreF32 {
+  struct Params {
+    float* y;
+    int ldy;
+    int ncols;
+  };
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
+                                             int*) {
+    const bool valid = row < m_rows;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32(taddr + c * 32, r);
+      tmem_wait_ld();
+      const int col0 = nb * BN + c * 32;
+      if (valid && col0 < p.ncols) {
+        float* dst = p.y + static_cast<int64_t>(row) * p.ldy + col0;
+        if (col0 + 32 <= p.ncols) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            reinterpret_cast<float4*>(dst)[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < p.ncols - col0) dst[j] = __uint_as_float(r[j]);
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Overflow path, first stage: rows are dense-row slots r (< n_over).  The
+// accumulator holds x_m W_u for m = slot_row[r]; the epilogue multiplies by
+// the stored fp32 ReLU gate of that row where the tile overflowed and writes
+// zero elsewhere (those tiles are served from TwELL).  h is written as an
+// unevaluated sum of two bf16 numbers (hi + lo, |lo| <= 2^-9 |hi|) so that the
+// second stage keeps ~16 bits of h while feeding bf16 tensor cores.
+struct EpiOverflowProduct {
+  struct Params {
+    const uint16_t* counts;   // [M][N/T]
+    const float* dense_rows;  // [R_cap][N]
+    const int* slot_row;      // [R_cap]
+    uint16_t* h_over;         // [R_cap][2N]: bf16 hi part in columns [0, N), lo part in [N, 2N)
+    int N, T, C;
+  };
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
+                                             int*) {
+    const bool valid = row < m_rows;
+    const int m = valid ? p.slot_row[row] : -1;
+    const int NT = p.N / p.T;
+    const int t = (nb * BN) / p.T;
+    const bool ov = m >= 0 && p.counts[static_cast<int64_t>(m) * NT + t] > p.C;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t u[32];
+      tmem_ld_32x32(taddr + c * 32, u);
+      tmem_wait_ld();
+      if (valid) {
+        const int64_t off = static_cast<int64_t>(row) * p.N + nb * BN + c * 32;
+        uint4* dst_hi = reinterpret_cast<uint4*>(p.h_over + static_cast<int64_t>(row) * 2 * p.N + nb * BN + c * 32);
+        uint4* dst_lo = dst_hi + p.N / 8;
+        const float4* gsrc = reinterpret_cast<const float4*>(p.dense_rows + off);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          float h[8];
+          if (ov) {
+            const float4 g0 = gsrc[2 * v], g1 = gsrc[2 * v + 1];
+            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h[e] = __uint_as_float(u[8 * v + e]) * g[e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h[e] = 0.f;
+          }
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hi[e] = pack_bf16x2(h[2 * e], h[2 * e + 1]);
+            lo[e] = pack_bf16x2(h[2 * e] - __uint_as_float(hi[e] << 16),
+                                h[2 * e + 1] - __uint_as_float(hi[e] & 0xFFFF0000u));
+          }
+          dst_hi[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          dst_lo[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Overflow path, second stage: y[slot_row[r]][col] += acc.
+struct EpiAccumulateRows {
+  struct Params {
+    float* y;
+    const int* slot_row;
+    int ldy;
+    int ncols;
+  };
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
+                                             int*) {
+    const int m = row < m_rows ? p.slot_row[row] : -1;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32(taddr + c * 32, r);
+      tmem_wait_ld();
+      const int col0 = nb * BN + c * 32;
+      if (m >= 0 && col0 < p.ncols) {
+        float* dst = p.y + static_cast<int64_t>(m) * p.ldy + col0;
+        if (col0 + 32 <= p.ncols) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            float4 a = reinterpret_cast<float4*>(dst)[v];
+            a.x += __uint_as_float(r[4 * v]);
+            a.y += __uint_as_float(r[4 * v + 1]);
+            a.z += __uint_as_float(r[4 * v + 2]);
+            a.w += __uint_as_float(r[4 * v + 3]);
+            reinterpret_cast<float4*>(dst)[v] = a;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < p.ncols - col0) dst[j] += __uint_as_float(r[j]);
+        }
+      }
+    }
+  }
+};
+
+}  // namespace twell

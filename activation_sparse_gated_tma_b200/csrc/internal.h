@@ -1,0 +1,33 @@
+// Internal launch interface between the C ABI (twell_api.cu) and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "epilogues.cuh"
+#include "tc_gemm.cuh"
+
+namespace twell {
+
+// Gate GEMM (tile width T = 128 or 256) with the ReLU + TwELL epilogue.
+cudaError_t launch_gate_twell(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
+                              const EpiGateTwell::Params& p, int* ctrl, int grid, cudaStream_t s);
+// h = (x W_u) * ReLU(x W_g), bf16, BN = 128.
+cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
+                                 const GemmGeom& g, const EpiGatedProduct::Params& p, int* ctrl, int grid,
+                                 cudaStream_t s);
+// y = h W_d (W_d stored [N][K], read MN-major), fp32 store, BN = 256.
+cudaError_t launch_down_store(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const GemmGeom& g,
+                              const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s);
+// Overflow rows: h_over = (x_over W_u) * dense_rows on overflow tiles, BN = 128.
+cudaError_t launch_overflow_product(const CUtensorMap& tm_xo, const CUtensorMap& tm_wu, const GemmGeom& g,
+                                    const EpiOverflowProduct::Params& p, int* ctrl, int grid, cudaStream_t s);
+// Overflow rows: y[slot_row[r]] += h_over[r] W_d, BN = 256.
+cudaError_t launch_overflow_down(const CUtensorMap& tm_ho, const CUtensorMap& tm_wd, const GemmGeom& g,
+                                 const EpiAccumulateRows::Params& p, int* ctrl, int grid, cudaStream_t s);
+
+constexpr int kGateGroupM = 16;
+
+}  // namespace twell

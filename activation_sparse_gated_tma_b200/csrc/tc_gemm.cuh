@@ -1,0 +1,206 @@
+// Persistent tcgen05 GEMM engine for sm_100a.
+//
+//   D[m][n] = sum_k A[m][k] * B[n][k]      (B K-major:  B stored [N][K] row-major)
+//   D[m][n] = sum_k A[m][k] * B[k][n]      (B MN-major: B stored [K][N] row-major)
+//
+// A is always K-major ([M][K] row-major bf16).  DUAL runs a second B operand
+// through the same A tile into a second accumulator (used for gate+up).
+//
+// One CTA per SM, 192 threads:
+//   warp 0      TMA producer (one elected lane) filling a STAGES-deep smem ring
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: thread i of warp w owns TMEM lane 32*(w%4)+i, i.e.
+//               one output row of the 128-row tile, and runs Epi::run on it.
+// Accumulators are double-buffered in TMEM so the epilogue of tile i overlaps
+// the MMAs of tile i+1.  Every wait is bounded (see mbar_wait).
+#pragma once
+
+#include <cuda.h>
+
+#include "ptx.cuh"
+
+namespace twell {
+
+constexpr int kBM = 128;      // UMMA M (rows per tile, = TMEM lanes)
+constexpr int kBK = 64;       // bf16 elements per 128-byte swizzle row
+constexpr int kUmmaK = 16;    // K per tcgen05.mma kind::f16
+constexpr int kGemmThreads = 192;
+
+struct GemmGeom {
+  int M;                    // rows of A and D
+  int N;                    // columns of D
+  int K;                    // reduction length (multiple of kBK)
+  const int* m_limit;       // optional: only rows < min(M, *m_limit) are computed
+  int group_m;              // rasterisation: tiles walk group_m row blocks per column sweep
+  int b_k_wrap;             // if > 0, B's k-block index is kb % b_k_wrap (A = [A0 | A1] against B twice)
+};
+
+template <int BN, bool DUAL>
+struct GemmSmem {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes * (DUAL ? 2 : 1);
+  static constexpr int kAccCols = BN * (DUAL ? 2 : 1);
+  static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64 : (2 * kAccCols <= 128) ? 128 : (2 * kAccCols <= 256) ? 256 : 512;
+  static_assert(2 * kAccCols <= 512, "two accumulators must fit in TMEM");
+  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte swizzle-atom alignment");
+};
+
+template <int BN, bool DUAL, int STAGES>
+constexpr size_t gemm_smem_bytes() {
+  return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * GemmSmem<BN, DUAL>::kStageBytes +
+         (2 * STAGES + 4) * sizeof(uint64_t) + 16;
+}
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * num_n;
+  const int grp = tile / per_group;
+  const int first_m = grp * group_m;
+  const int gm = min(group_m, num_m - first_m);
+  const int r = tile - grp * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+template <int BN, bool B_MN, bool DUAL, int STAGES, class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, const GemmGeom g, const typename Epi::Params ep,
+                   int* ctrl) {
+  using L = GemmSmem<BN, DUAL>;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "UMMA N for M=128 must be a multiple of 16 up to 256");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  int m_rows = g.M;
+  if (g.m_limit) m_rows = min(m_rows, *g.m_limit);
+  const int num_m = (m_rows + kBM - 1) / kBM;
+  const int num_n = (g.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = g.K / kBK;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0 && num_tiles > blockIdx.x) {
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      if (DUAL) prefetch_tmap(&tmB2);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, g.group_m, mb, nb);
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, ctrl)) { ok = false; break; }
+          uint8_t* sa = smem + stage * L::kStageBytes;
+          uint8_t* sb = sa + L::kABytes;
+          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          tma_load_2d(&tmA, &full[stage], sa, kb * kBK, mb * kBM);
+          const int kbb = g.b_k_wrap > 0 ? kb % g.b_k_wrap : kb;
+          if (!B_MN) {
+            tma_load_2d(&tmB, &full[stage], sb, kbb * kBK, nb * BN);
+            if (DUAL) tma_load_2d(&tmB2, &full[stage], sb + L::kBBytes, kbb * kBK, nb * BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) {
+              tma_load_2d(&tmB, &full[stage], sb + j * 8192, nb * BN + j * 64, kbb * kBK);
+              if (DUAL) tma_load_2d(&tmB2, &full[stage], sb + L::kBBytes + j * 8192, nb * BN + j * 64, kbb * kBK);
+            }
+          }
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, ctrl)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * L::kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, ctrl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * L::kStageBytes);
+          const uint32_t b_base = a_base + L::kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bdesc = B_MN ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+                                        : smem_desc_sw128(b_base + k * 32, 16, 1024);
+            const uint32_t accum = (kb | k) != 0;
+            umma_bf16(d, adesc, bdesc, idesc, accum);
+            if (DUAL) {
+              const uint32_t b2 = b_base + L::kBBytes;
+              const uint64_t bdesc2 =
+                  B_MN ? smem_desc_sw128(b2 + k * 2048, 8192, 1024) : smem_desc_sw128(b2 + k * 32, 16, 1024);
+              umma_bf16(d + BN, adesc, bdesc2, idesc, accum);
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, g.group_m, mb, nb);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, ctrl)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
+      Epi::template run<BN>(ep, taddr, mb * kBM + row_in_tile, m_rows, nb, lane, ctrl);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, L::kTmemCols);
+}
+
+}  // namespace twell

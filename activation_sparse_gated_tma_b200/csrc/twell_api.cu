@@ -1,0 +1,377 @@
+// C ABI of the sparse gated FFN forward path (declared in include/twell.h).
+// Host side only does validation, TMA descriptor encoding and launches;
+// every arithmetic step runs in the kernels.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "../../include/twell.h"
+#include "internal.h"
+#include "sparse_updown.cuh"
+
+namespace twell {
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local int g_launches = 0;
+
+twell_status fail(twell_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define TW_CUDA(expr)                                                                              \
+  do {                                                                                             \
+    cudaError_t e_ = (expr);                                                                       \
+    if (e_ != cudaSuccess) return fail(TWELL_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- device info
+struct DeviceInfo {
+  int sms = 0;
+  int cc_major = 0;
+};
+
+twell_status device_info(DeviceInfo& info) {
+  int dev = 0;
+  TW_CUDA(cudaGetDevice(&dev));
+  static std::mutex mu;
+  static std::map<int, DeviceInfo> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
+    DeviceInfo d;
+    TW_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    TW_CUDA(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+    it = cache.emplace(dev, d).first;
+  }
+  info = it->second;
+  if (info.cc_major != 10) return fail(TWELL_ERR_UNSUPPORTED, "needs an sm_100 device (found cc %d.x)", info.cc_major);
+  return TWELL_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 row-major [outer][inner] matrix, box [box_outer][64], 128-byte swizzle,
+// zero fill out of bounds.  Cached by (device, pointer, shape, box).
+twell_status tmap_bf16(const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer, CUtensorMap& out) {
+  using Key = std::tuple<int, uintptr_t, uint64_t, uint64_t, uint32_t>;
+  static std::mutex mu;
+  static std::map<Key, CUtensorMap> cache;
+  int dev = 0;
+  TW_CUDA(cudaGetDevice(&dev));
+  const Key key{dev, reinterpret_cast<uintptr_t>(ptr), inner, outer, box_outer};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      out = it->second;
+      return TWELL_OK;
+    }
+  }
+  auto enc = encode_fn();
+  if (!enc) return fail(TWELL_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TWELL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() > 4096) cache.clear();
+  cache.emplace(key, out);
+  return TWELL_OK;
+}
+
+// ---------------------------------------------------------------- buffer layout
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Layout {
+  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, total;
+};
+
+bool shape_ok(int M, int K, int N, int T, int C, int R_cap) {
+  return M >= 1 && K >= 64 && K <= 4096 && K % 64 == 0 && (T == 128 || T == 256) && N >= T && N % T == 0 &&
+         C >= 1 && C <= T && C <= 255 && R_cap >= 1 && static_cast<int64_t>(M) * N < (int64_t(1) << 40);
+}
+
+Layout layout(int M, int K, int N, int T, int C, int R_cap) {
+  const size_t NT = static_cast<size_t>(N / T);
+  Layout L;
+  size_t o = 0;
+  L.ctrl = o; o = align256(o + kCtrlWords * sizeof(int));
+  L.counts = o; o = align256(o + size_t(M) * NT * 2);
+  L.idx = o; o = align256(o + size_t(M) * NT * C);
+  L.vals = o; o = align256(o + size_t(M) * NT * C * 4);
+  L.row_slot = o; o = align256(o + size_t(M) * 4);
+  L.slot_row = o; o = align256(o + size_t(R_cap) * 4);
+  L.dense_rows = o; o = align256(o + size_t(R_cap) * N * 4);
+  L.x_over = o; o = align256(o + size_t(R_cap) * K * 2);
+  L.h_over = o; o = align256(o + size_t(R_cap) * N * 4);
+  L.total = o;
+  return L;
+}
+
+twell_status check_buf(const twell_buf* tw) {
+  if (!tw) return fail(TWELL_ERR_INVALID, "twell_buf is NULL");
+  if (!shape_ok(tw->M, tw->K, tw->N, tw->T, tw->C, tw->R_cap)) return fail(TWELL_ERR_INVALID, "twell_buf has invalid sizes");
+  if (!tw->counts || !tw->idx || !tw->vals || !tw->dense_rows || !tw->row_slot || !tw->slot_row || !tw->ctrl ||
+      !tw->x_over || !tw->h_over)
+    return fail(TWELL_ERR_INVALID, "twell_buf is not initialised");
+  return TWELL_OK;
+}
+
+// ---------------------------------------------------------------- small kernels
+// Start of a gate pass: no row holds a dense-row slot, control words at zero.
+__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < kCtrlWords) ctrl[i] = 0;
+  for (int r = i; r < M; r += gridDim.x * blockDim.x) row_slot[r] = kSlotFree;
+}
+
+// Warps per CTA and ring depth of the fused kernel for a given K: eight warps
+// when each can keep at least two entries in flight, else four.
+void updown_config(int K, int& warps, int& stages) {
+  constexpr size_t kBudget = 232448;  // 227 KB of dynamic shared memory per CTA
+  for (warps = 8; warps >= 4; warps /= 2) {
+    const size_t per_warp = kBudget / warps;
+    const size_t fixed = kUpdownListCap * 8 + 128;
+    stages = per_warp > fixed ? static_cast<int>((per_warp - fixed) / (4 * static_cast<size_t>(K) + 8)) : 0;
+    if (stages > 8) stages = 8;
+    if (stages >= 2) return;
+  }
+  warps = 4;
+}
+
+template <int KV>
+cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
+                             float* y, int sms, cudaStream_t s) {
+  int warps = 8, stages = 2;
+  updown_config(tw->K, warps, stages);
+  if (stages < 1) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(warps) * updown_warp_bytes(tw->K, stages);
+  cudaError_t e = cudaFuncSetAttribute(twell_updown_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int rows_per_wave = warps;
+  int grid = sms;
+  const int max_grid = (tw->M + rows_per_wave - 1) / rows_per_wave;
+  if (grid > max_grid) grid = max_grid;
+  twell_updown_kernel<KV><<<grid, 32 * warps, smem, s>>>(x, wu_t, wd, tw->counts, tw->idx, tw->vals, tw->M, tw->K,
+                                                        tw->N, tw->T, tw->C, y, tw->ctrl, stages);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_updown(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw, float* y,
+                          int sms, cudaStream_t s) {
+  switch ((tw->K + 255) / 256) {
+#define TW_KV(n) \
+  case n:        \
+    return launch_updown_kv<n>(x, wu_t, wd, tw, y, sms, s);
+    TW_KV(1) TW_KV(2) TW_KV(3) TW_KV(4) TW_KV(5) TW_KV(6) TW_KV(7) TW_KV(8)
+    TW_KV(9) TW_KV(10) TW_KV(11) TW_KV(12) TW_KV(13) TW_KV(14) TW_KV(15) TW_KV(16)
+#undef TW_KV
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+int gemm_grid(int rows, int cols, int bn, int sms) {
+  const long tiles = static_cast<long>((rows + kBM - 1) / kBM) * ((cols + bn - 1) / bn);
+  return static_cast<int>(tiles < sms ? tiles : sms);
+}
+
+}  // namespace
+}  // namespace twell
+
+using namespace twell;
+
+extern "C" {
+
+const char* twell_status_str(twell_status st) {
+  switch (st) {
+    case TWELL_OK: return "ok";
+    case TWELL_ERR_INVALID: return "invalid argument";
+    case TWELL_ERR_CAPACITY: return "dense-row capacity exceeded";
+    case TWELL_ERR_CUDA: return "CUDA error";
+    case TWELL_ERR_DEVICE_CHECK: return "device status flag raised";
+    case TWELL_ERR_UNSUPPORTED: return "unsupported device or shape";
+  }
+  return "unknown status";
+}
+
+const char* twell_last_error(void) { return g_err; }
+
+int twell_last_launch_count(void) { return g_launches; }
+
+size_t twell_buf_bytes(int M, int K, int N, int T, int C, int R_cap) {
+  if (!shape_ok(M, K, N, T, C, R_cap)) return 0;
+  return layout(M, K, N, T, C, R_cap).total;
+}
+
+twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int K, int N, int T, int C, int R_cap) {
+  g_launches = 0;
+  if (!tw) return fail(TWELL_ERR_INVALID, "twell_buf is NULL");
+  if (!shape_ok(M, K, N, T, C, R_cap))
+    return fail(TWELL_ERR_INVALID, "invalid sizes M=%d K=%d N=%d T=%d C=%d R_cap=%d", M, K, N, T, C, R_cap);
+  if (!base || (reinterpret_cast<uintptr_t>(base) & 255u)) return fail(TWELL_ERR_INVALID, "base must be 256-byte aligned");
+  const Layout L = layout(M, K, N, T, C, R_cap);
+  if (bytes < L.total) return fail(TWELL_ERR_INVALID, "buffer too small: %zu < %zu bytes", bytes, L.total);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  tw->ctrl = reinterpret_cast<int32_t*>(b + L.ctrl);
+  tw->counts = reinterpret_cast<uint16_t*>(b + L.counts);
+  tw->idx = b + L.idx;
+  tw->vals = reinterpret_cast<float*>(b + L.vals);
+  tw->row_slot = reinterpret_cast<int32_t*>(b + L.row_slot);
+  tw->slot_row = reinterpret_cast<int32_t*>(b + L.slot_row);
+  tw->dense_rows = reinterpret_cast<float*>(b + L.dense_rows);
+  tw->x_over = reinterpret_cast<uint16_t*>(b + L.x_over);
+  tw->h_over = reinterpret_cast<uint16_t*>(b + L.h_over);
+  tw->M = M; tw->K = K; tw->N = N; tw->T = T; tw->C = C; tw->R_cap = R_cap;
+  return TWELL_OK;
+}
+
+twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int K, int N, twell_buf* tw,
+                             int* n_over_host, cudaStream_t stream) {
+  g_launches = 0;
+  twell_status st = check_buf(tw);
+  if (st != TWELL_OK) return st;
+  if (M != tw->M || K != tw->K || N != tw->N)
+    return fail(TWELL_ERR_INVALID, "shape (%d,%d,%d) does not match the buffer (%d,%d,%d)", M, K, N, tw->M, tw->K, tw->N);
+  if (!aligned16(x) || !aligned16(wg_t)) return fail(TWELL_ERR_INVALID, "x and wg_t must be non-NULL and 16-byte aligned");
+  DeviceInfo dev;
+  if ((st = device_info(dev)) != TWELL_OK) return st;
+
+  CUtensorMap tm_x, tm_wg;
+  if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wg_t, K, N, tw->T, tm_wg)) != TWELL_OK) return st;
+
+  const int rgrid = static_cast<int>((static_cast<int64_t>(M) + 255) / 256 < 1024 ? (M + 255) / 256 : 1024);
+  twell_reset_kernel<<<rgrid > 0 ? rgrid : 1, 256, 0, stream>>>(tw->row_slot, M, tw->ctrl);
+  TW_CUDA(cudaGetLastError());
+  ++g_launches;
+
+  EpiGateTwell::Params p;
+  p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.dense_rows = tw->dense_rows;
+  p.row_slot = tw->row_slot; p.slot_row = tw->slot_row; p.x = x; p.x_over = tw->x_over;
+  p.N = N; p.K = K; p.C = tw->C; p.r_cap = tw->R_cap;
+  GemmGeom g{M, N, K, nullptr, kGateGroupM, 0};
+  TW_CUDA(launch_gate_twell(tw->T, tm_x, tm_wg, g, p, tw->ctrl, gemm_grid(M, N, tw->T, dev.sms), stream));
+  ++g_launches;
+
+  if (n_over_host) {
+    int n_over = 0;
+    int flags = 0;
+    if ((st = twell_read_status(tw, &n_over, &flags, stream)) == TWELL_ERR_DEVICE_CHECK) return st;
+    *n_over_host = n_over;
+    if (n_over > tw->R_cap)
+      return fail(TWELL_ERR_CAPACITY, "%d rows overflowed, dense-row capacity is %d", n_over, tw->R_cap);
+  }
+  return TWELL_OK;
+}
+
+twell_status twell_read_status(const twell_buf* tw, int* n_over_host, int* device_flags, cudaStream_t stream) {
+  twell_status st = check_buf(tw);
+  if (st != TWELL_OK) return st;
+  int words[2] = {0, 0};
+  TW_CUDA(cudaMemcpyAsync(words, tw->ctrl, sizeof words, cudaMemcpyDeviceToHost, stream));
+  TW_CUDA(cudaStreamSynchronize(stream));
+  if (n_over_host) *n_over_host = words[kCtrlNOver];
+  if (device_flags) *device_flags = words[kCtrlFlags];
+  if (words[kCtrlFlags] & ~kFlagNoCapacity)
+    return fail(TWELL_ERR_DEVICE_CHECK, "device status flags 0x%x", words[kCtrlFlags]);
+  if (words[kCtrlNOver] > tw->R_cap)
+    return fail(TWELL_ERR_CAPACITY, "%d rows overflowed, dense-row capacity is %d", words[kCtrlNOver], tw->R_cap);
+  return TWELL_OK;
+}
+
+twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw, int K,
+                           float* y, cudaStream_t stream) {
+  g_launches = 0;
+  twell_status st = check_buf(tw);
+  if (st != TWELL_OK) return st;
+  if (K != tw->K) return fail(TWELL_ERR_INVALID, "K=%d does not match the buffer's K=%d", K, tw->K);
+  if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y))
+    return fail(TWELL_ERR_INVALID, "x, wu_t, wd and y must be non-NULL and 16-byte aligned");
+  DeviceInfo dev;
+  if ((st = device_info(dev)) != TWELL_OK) return st;
+  const int N = tw->N;
+
+  TW_CUDA(launch_updown(x, wu_t, wd, tw, y, dev.sms, stream));
+  ++g_launches;
+
+  // Dense-row path for overflow tiles; rows beyond the device-side n_over are skipped.
+  CUtensorMap tm_xo, tm_wu, tm_ho, tm_wd;
+  if ((st = tmap_bf16(tw->x_over, K, tw->R_cap, kBM, tm_xo)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wu_t, K, N, 128, tm_wu)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(tw->h_over, 2 * N, tw->R_cap, kBM, tm_ho)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wd, K, N, 64, tm_wd)) != TWELL_OK) return st;
+
+  EpiOverflowProduct::Params p1;
+  p1.counts = tw->counts; p1.dense_rows = tw->dense_rows; p1.slot_row = tw->slot_row; p1.h_over = tw->h_over;
+  p1.N = N; p1.T = tw->T; p1.C = tw->C;
+  GemmGeom g1{tw->R_cap, N, K, tw->ctrl + kCtrlNOver, kGateGroupM, 0};
+  TW_CUDA(launch_overflow_product(tm_xo, tm_wu, g1, p1, tw->ctrl, gemm_grid(tw->R_cap, N, 128, dev.sms), stream));
+  ++g_launches;
+
+  EpiAccumulateRows::Params p2;
+  p2.y = y; p2.slot_row = tw->slot_row; p2.ldy = K; p2.ncols = K;
+  GemmGeom g2{tw->R_cap, K, 2 * N, tw->ctrl + kCtrlNOver, kGateGroupM, N / kBK};
+  TW_CUDA(launch_overflow_down(tm_ho, tm_wd, g2, p2, tw->ctrl, gemm_grid(tw->R_cap, K, 256, dev.sms), stream));
+  ++g_launches;
+  return TWELL_OK;
+}
+
+twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd, int M,
+                           int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream) {
+  g_launches = 0;
+  if (M < 1 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0)
+    return fail(TWELL_ERR_INVALID, "invalid sizes M=%d K=%d N=%d (need K %% 64 == 0, N %% 128 == 0)", M, K, N);
+  if (!aligned16(x) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(h_scratch) || !aligned16(y))
+    return fail(TWELL_ERR_INVALID, "all pointers must be non-NULL and 16-byte aligned");
+  twell_status st;
+  DeviceInfo dev;
+  if ((st = device_info(dev)) != TWELL_OK) return st;
+  CUtensorMap tm_x, tm_wg, tm_wu, tm_h, tm_wd;
+  if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wg_t, K, N, 128, tm_wg)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wu_t, K, N, 128, tm_wu)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(h_scratch, N, M, kBM, tm_h)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wd, K, N, 64, tm_wd)) != TWELL_OK) return st;
+
+  EpiGatedProduct::Params p1{h_scratch, N};
+  GemmGeom g1{M, N, K, nullptr, kGateGroupM, 0};
+  TW_CUDA(launch_gated_product(tm_x, tm_wg, tm_wu, g1, p1, nullptr, gemm_grid(M, N, 128, dev.sms), stream));
+  ++g_launches;
+  EpiStoreF32::Params p2{y, K, K};
+  GemmGeom g2{M, K, N, nullptr, kGateGroupM, 0};
+  TW_CUDA(launch_down_store(tm_h, tm_wd, g2, p2, nullptr, gemm_grid(M, K, 256, dev.sms), stream));
+  ++g_launches;
+  return TWELL_OK;
+}
+
+}  // extern "C"

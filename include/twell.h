@@ -1,0 +1,161 @@
+/*
+ * twell.h - C ABI of the B200 (sm_100a) ReLU-gated sparse FFN forward path.
+ *
+ * The operation ("Sparser, Faster, Lighter Transformer Language Models",
+ * review page dimensionstp.github.io, §1-1 problem definition):
+ *
+ *     h_u = x W_u,   h_g = ReLU(x W_g),   h = h_u (.) h_g,   y = h W_d
+ *
+ * with x [M x K] tokens, W_g and W_u mapping K -> N, W_d mapping N -> K.
+ * The sparse path computes it in two steps (§2-2, §3-4, §3-5):
+ *   twell_gate_pack : gate GEMM on tensor cores whose epilogue applies ReLU and
+ *                     packs every row's non-zeros tile-locally into TwELL
+ *                     (Tile-wise ELLPACK), never writing the dense gate;
+ *   twell_ffn_fwd   : fused up + down projection that visits only the active
+ *                     hidden units: y_m = sum_{n in A_m} g_{m,n} (x_m W_u[:,n]) W_d[n,:].
+ * Tiles whose active count exceeds the capacity C are routed to a dense-row
+ * backup (§3-6 hybrid format; §4-3 static capacity of at most M/8 rows,
+ * overflow reported to the host, which retries with larger storage).
+ * dense_ffn_fwd computes the same y with dense tensor-core GEMMs.
+ *
+ * Conventions for every entry point:
+ *   - bf16 tensors are passed as uint16_t bit patterns; all matrices are
+ *     row-major and contiguous; every pointer must be 16-byte aligned.
+ *   - All device pointers are owned by the caller.  The library allocates no
+ *     device memory and keeps no state except cached TMA descriptors (keyed by
+ *     pointer and shape) and per-device kernel attributes.
+ *   - Work is enqueued on `stream` and is asynchronous unless stated.
+ *   - Invalid arguments return TWELL_ERR_INVALID before anything is launched.
+ *   - A failing CUDA call returns TWELL_ERR_CUDA (message: twell_last_error()).
+ *
+ * Weight layouts (N rows of K, so each hidden unit n is one contiguous row):
+ *   wg_t[n][k] = W_g[k][n],  wu_t[n][k] = W_u[k][n],  wd[n][k] = W_d[n][k].
+ * The gate bias, if any, rides in the GEMM (x[:,K-1] = 1, wg_t[:,K-1] = -b).
+ */
+#ifndef TWELL_H_
+#define TWELL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TWELL_OK = 0,
+  TWELL_ERR_INVALID = 1,      /* bad shape, pointer, alignment or buffer; nothing launched */
+  TWELL_ERR_CAPACITY = 2,     /* more rows overflowed than the dense-row buffer holds */
+  TWELL_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  TWELL_ERR_DEVICE_CHECK = 4, /* a kernel raised a device status flag (bounded wait expired) */
+  TWELL_ERR_UNSUPPORTED = 5   /* no sm_100 device, or a shape outside the kernels' limits */
+} twell_status;
+
+/*
+ * TwELL activations plus the hybrid dense-row backup, all in one caller-owned
+ * device block carved by twell_buf_init.  Sizes: NT = N / T.
+ *
+ *   counts     uint16 [M][NT]     true number of active units (z > 0) of row m
+ *                                 in column tile t; a count > C marks the tile
+ *                                 as overflow (its slots are then not used)
+ *   idx        uint8  [M][NT][C]  local index n - t*T of the first min(count, C)
+ *                                 active units, ascending; later slots undefined
+ *   vals       fp32   [M][NT][C]  ReLU(z) of those units (the fp32 GEMM result)
+ *   dense_rows fp32   [R_cap][N]  ReLU(z) of the overflow tiles of the row that
+ *                                 owns the slot; other tiles of the slot undefined
+ *   row_slot   int32  [M]         dense-row slot of row m; -1 = none;
+ *                                 -2 = needed but R_cap was exhausted
+ *   slot_row   int32  [R_cap]     row that owns each slot (valid for slots < n_over)
+ *   ctrl       int32  [64]        device control words: [0] n_over (rows that
+ *                                 asked for a slot), [1] status flags, [2..3]
+ *                                 work-queue counters
+ *   x_over     bf16   [R_cap][K]  scratch: gathered x rows of slotted rows
+ *   h_over     bf16   [R_cap][2N] scratch: overflow-tile hidden activations as
+ *                                 bf16 hi (columns < N) + lo (columns >= N) parts
+ */
+typedef struct twell_buf {
+  uint16_t* counts;
+  uint8_t* idx;
+  float* vals;
+  float* dense_rows;
+  int32_t* row_slot;
+  int32_t* slot_row;
+  int32_t* ctrl;
+  uint16_t* x_over;
+  uint16_t* h_over;
+  int M, K, N, T, C, R_cap;
+} twell_buf;
+
+/* Bytes of device memory twell_buf_init needs for these sizes (0 if invalid). */
+size_t twell_buf_bytes(int M, int K, int N, int T, int C, int R_cap);
+
+/*
+ * Carve `base` (device pointer, >= twell_buf_bytes(...) bytes, 256-byte
+ * aligned) into the arrays of `tw`.  Host-side pointer arithmetic only; the
+ * contents are initialised by twell_gate_pack.  Limits: M >= 1, K % 64 == 0,
+ * 64 <= K <= 4096, T in {128, 256}, N % T == 0, 1 <= C <= min(T, 255),
+ * 1 <= R_cap.
+ */
+twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int K, int N, int T, int C,
+                            int R_cap);
+
+/*
+ * Gate GEMM + ReLU + TwELL pack + overflow routing (one launch after a small
+ * reset kernel).  x [M][K], wg_t [N][K] device bf16.  M, K, N must equal the
+ * buffer's.  Fills every array of `tw` described above.
+ *
+ * n_over_host: if NULL the call is fully asynchronous; the overflow count stays
+ * on the device (ctrl[0]) and twell_read_status reports it later.  If not NULL
+ * the call synchronises `stream`, stores the number of rows that asked for a
+ * dense-row slot and returns TWELL_ERR_CAPACITY when it exceeds R_cap; the
+ * caller then re-initialises a buffer with R_cap >= *n_over_host and calls
+ * again (the pages' CPU-side flag and retry).
+ */
+twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int K, int N, twell_buf* tw,
+                             int* n_over_host, cudaStream_t stream);
+
+/*
+ * Fused sparse up + down projection over `tw` (filled by twell_gate_pack on the
+ * same stream), then the dense-row path for overflow tiles.  wu_t, wd [N][K]
+ * device bf16; y [M][K] device fp32, fully overwritten.  K must equal tw->K.
+ * Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
+ * -2 in row_slot miss their overflow tiles and twell_read_status returns
+ * TWELL_ERR_CAPACITY.
+ */
+twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
+                           int K, float* y, cudaStream_t stream);
+
+/*
+ * Synchronises `stream` and reads the buffer's device control words.
+ * Returns TWELL_ERR_DEVICE_CHECK if a device status flag other than the
+ * capacity flag is set, else TWELL_ERR_CAPACITY if n_over > R_cap, else
+ * TWELL_OK.  Either output pointer may be NULL.
+ */
+twell_status twell_read_status(const twell_buf* tw, int* n_over_host, int* device_flags, cudaStream_t stream);
+
+/*
+ * Dense comparison FFN (§1-1 computed in full, §2-2 "dense pipeline"):
+ * GEMM 1 computes x W_g and x W_u for the same column tile into two TMEM
+ * accumulators and writes h = (x W_u) * ReLU(x W_g) as bf16 into h_scratch
+ * [M][N] (device, caller-owned); GEMM 2 writes y = h W_d, fp32 [M][K].
+ * Limits: K % 64 == 0, N % 128 == 0.  Asynchronous.
+ */
+twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
+                           int M, int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* twell_status_str(twell_status status);
+
+/* Message of the last TWELL_ERR_CUDA / TWELL_ERR_INVALID on this thread. */
+const char* twell_last_error(void);
+
+/* Number of kernels the last call on this thread enqueued (for launch accounting). */
+int twell_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TWELL_H_ */

@@ -1,0 +1,102 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function include/twell.h declares, and rejects invalid arguments before it
+touches CUDA."""
+import ctypes
+
+import pytest
+
+from activation_sparse_gated_tma_b200 import twell as tw
+
+
+def test_library_exports_every_header_function():
+    L = tw.lib()
+    names = tw.header_functions()
+    assert {"twell_gate_pack", "twell_ffn_fwd", "dense_ffn_fwd"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    L = tw.lib()
+    for s in range(6):
+        assert L.twell_status_str(s)
+    assert L.twell_status_str(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("args", [
+    (0, 256, 1024, 128, 8, 1),      # M < 1
+    (64, 200, 1024, 128, 8, 1),     # K % 64
+    (64, 8192, 1024, 128, 8, 1),    # K > 4096
+    (64, 256, 1000, 128, 8, 1),     # N % T
+    (64, 256, 1024, 64, 8, 1),      # T not in {128, 256}
+    (64, 256, 1024, 128, 0, 1),     # C < 1
+    (64, 256, 1024, 128, 129, 1),   # C > T
+    (64, 256, 1024, 128, 8, 0),     # R_cap < 1
+])
+def test_buf_bytes_rejects_invalid_sizes(args):
+    assert tw.lib().twell_buf_bytes(*args) == 0
+
+
+def test_buf_init_layout_is_aligned_and_disjoint():
+    L = tw.lib()
+    M, K, N, T, C, R = 100, 256, 1024, 128, 8, 13
+    nbytes = L.twell_buf_bytes(M, K, N, T, C, R)
+    assert nbytes > 0
+    base = 1 << 32                      # host-side pointer arithmetic only; never dereferenced
+    b = tw._TwellBuf()
+    assert L.twell_buf_init(ctypes.byref(b), base, nbytes, M, K, N, T, C, R) == tw.OK
+    NT = N // T
+    spans = [("ctrl", 64 * 4), ("counts", M * NT * 2), ("idx", M * NT * C), ("vals", M * NT * C * 2),
+             ("row_slot", M * 4), ("slot_row", R * 4), ("dense_rows", R * N * 2), ("x_over", R * K * 2),
+             ("h_over", R * N * 2)]
+    ranges = []
+    for name, size in spans:
+        p = getattr(b, name)
+        assert p % 256 == 0
+        assert base <= p and p + size <= base + nbytes
+        ranges.append((p, p + size))
+    ranges.sort()
+    assert all(a[1] <= c[0] for a, c in zip(ranges, ranges[1:]))
+    assert (b.M, b.K, b.N, b.T, b.C, b.R_cap) == (M, K, N, T, C, R)
+    # too small / misaligned
+    assert L.twell_buf_init(ctypes.byref(b), base, nbytes - 1, M, K, N, T, C, R) == tw.ERR_INVALID
+    assert L.twell_buf_init(ctypes.byref(b), base + 16, nbytes, M, K, N, T, C, R) == tw.ERR_INVALID
+    assert b"aligned" in L.twell_last_error()
+
+
+def _fake_buf():
+    L = tw.lib()
+    M, K, N, T, C, R = 64, 256, 1024, 128, 8, 8
+    b = tw._TwellBuf()
+    assert L.twell_buf_init(ctypes.byref(b), 1 << 32, L.twell_buf_bytes(M, K, N, T, C, R), M, K, N, T, C, R) == tw.OK
+    return b
+
+
+def test_gate_pack_validates_before_launch():
+    L = tw.lib()
+    b = _fake_buf()
+    x, w = 1 << 33, 1 << 34           # aligned fake device pointers: validation must fail before any use
+    assert L.twell_gate_pack(None, w, 64, 256, 1024, ctypes.byref(b), None, None) == tw.ERR_INVALID
+    assert L.twell_gate_pack(x + 8, w, 64, 256, 1024, ctypes.byref(b), None, None) == tw.ERR_INVALID
+    assert L.twell_gate_pack(x, w, 65, 256, 1024, ctypes.byref(b), None, None) == tw.ERR_INVALID
+    assert L.twell_gate_pack(x, w, 64, 256, 1024, None, None, None) == tw.ERR_INVALID
+    empty = tw._TwellBuf()
+    assert L.twell_gate_pack(x, w, 64, 256, 1024, ctypes.byref(empty), None, None) == tw.ERR_INVALID
+
+
+def test_ffn_fwd_and_dense_validate_before_launch():
+    L = tw.lib()
+    b = _fake_buf()
+    p = 1 << 33
+    assert L.twell_ffn_fwd(p, p, p, ctypes.byref(b), 128, p, None) == tw.ERR_INVALID     # K mismatch
+    assert L.twell_ffn_fwd(p, p, None, ctypes.byref(b), 256, p, None) == tw.ERR_INVALID
+    assert L.twell_ffn_fwd(p, p, p, ctypes.byref(b), 256, p + 4, None) == tw.ERR_INVALID
+    assert L.dense_ffn_fwd(p, p, p, p, 64, 200, 1024, p, p, None) == tw.ERR_INVALID      # K % 64
+    assert L.dense_ffn_fwd(p, p, p, p, 64, 256, 1000, p, p, None) == tw.ERR_INVALID      # N % 128
+    assert L.dense_ffn_fwd(p, p, p, p, 64, 256, 1024, None, p, None) == tw.ERR_INVALID
+
+
+def test_python_wrapper_rejects_wrong_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        tw._bf16(torch.zeros(4, 4), "x", (4, 4))          # wrong dtype / not CUDA
