@@ -8,6 +8,7 @@ a dense-row tensor-core path for tiles that overflow the TwELL capacity.
 """
 from .twell import (  # noqa: F401
     CapacityError,
+    KernelTrace,
     TwellBuffers,
     TwellError,
     dense_ffn,

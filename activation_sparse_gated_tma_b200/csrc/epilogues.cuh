@@ -51,78 +51,88 @@ __device__ __forceinline__ float relu_f(float z) { return z > 0.f ? z : 0.f; }
 // ---------------------------------------------------------------------------
 // Gate epilogue: ReLU + TwELL packing + overflow routing ("Sparser, Faster,
 // Lighter Transformer Language Models", §3-4 steps 3-5 and §3-6).
-// The tile width T equals BN, so a (row, tile) record is produced entirely by
-// one thread from its own TMEM lane: no cross-CTA or cross-thread step.
+// The CTA's output tile (BN columns) holds BN / T whole TwELL tiles, so every
+// (row, tile) record is produced by one thread from its own TMEM lane: no
+// cross-CTA or cross-thread step is needed to pack.
+struct GateTwellParams {
+  uint16_t* counts;    // [M][N/T]
+  uint8_t* idx;        // [M][N/T][C]
+  float* vals;         // [M][N/T][C]
+  float* dense_rows;   // [R_cap][N]
+  int* row_slot;       // [M]
+  int* slot_row;       // [R_cap]
+  const uint16_t* x;   // [M][K] gate input, copied to x_over for slotted rows
+  uint16_t* x_over;    // [R_cap][K]
+  int N, K, C, r_cap;
+};
+
+template <int T>
 struct EpiGateTwell {
-  struct Params {
-    uint16_t* counts;      // [M][N/T]
-    uint8_t* idx;          // [M][N/T][C]
-    float* vals;           // [M][N/T][C]
-    float* dense_rows;     // [R_cap][N]
-    int* row_slot;         // [M]
-    int* slot_row;         // [R_cap]
-    const uint16_t* x;     // [M][K] gate input, copied to x_over for slotted rows
-    uint16_t* x_over;      // [R_cap][K]
-    int N, K, C, r_cap;
-  };
+  using Params = GateTwellParams;
 
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb,
                                              int lane, int* ctrl) {
+    static_assert(BN % T == 0, "a CTA tile must hold whole TwELL tiles");
     const bool valid = row < m_rows;
-    const int NT = p.N / BN;
-    const int64_t rec = static_cast<int64_t>(row) * NT + nb;
-    uint8_t* idx_rec = p.idx + rec * p.C;
-    float* val_rec = p.vals + rec * p.C;
-    int cnt = 0;
+    const int NT = p.N / T;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld_32x32(taddr + c * 32, r);
-      tmem_wait_ld();
-      if (valid) {
+    for (int st = 0; st < BN / T; ++st) {
+      const int t = nb * (BN / T) + st;
+      const uint32_t tcol = taddr + st * T;
+      const int64_t rec = static_cast<int64_t>(row) * NT + t;
+      uint8_t* idx_rec = p.idx + rec * p.C;
+      float* val_rec = p.vals + rec * p.C;
+      int cnt = 0;
+#pragma unroll 1
+      for (int c = 0; c < T / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32(tcol + c * 32, r);
+        tmem_wait_ld();
+        if (valid) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float z = __uint_as_float(r[j]);
-          if (z > 0.f) {
-            if (cnt < p.C) {
-              idx_rec[cnt] = static_cast<uint8_t>(c * 32 + j);
-              val_rec[cnt] = z;
+          for (int j = 0; j < 32; ++j) {
+            const float z = __uint_as_float(r[j]);
+            if (z > 0.f) {
+              if (cnt < p.C) {
+                idx_rec[cnt] = static_cast<uint8_t>(c * 32 + j);
+                val_rec[cnt] = z;
+              }
+              ++cnt;
             }
-            ++cnt;
           }
         }
       }
-    }
-    if (valid) p.counts[rec] = static_cast<uint16_t>(cnt);
-    const bool ov = valid && cnt > p.C;
-    if (__any_sync(0xffffffffu, ov)) {
-      int slot = -1;
-      bool fresh = false;
-      if (ov) slot = acquire_row_slot(p.row_slot, p.slot_row, p.r_cap, row, ctrl, fresh);
-      // The lane that opened a slot brings its x row along (whole warp copies).
-      uint32_t fresh_mask = __ballot_sync(0xffffffffu, fresh);
-      while (fresh_mask) {
-        const int src = __ffs(fresh_mask) - 1;
-        fresh_mask &= fresh_mask - 1;
-        const int r = __shfl_sync(0xffffffffu, row, src);
-        const int sl = __shfl_sync(0xffffffffu, slot, src);
-        const uint4* xs = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.K);
-        uint4* xd = reinterpret_cast<uint4*>(p.x_over + static_cast<int64_t>(sl) * p.K);
-        for (int v = lane; v < p.K / 8; v += 32) xd[v] = xs[v];
-      }
-      float* dst = slot >= 0 ? p.dense_rows + static_cast<int64_t>(slot) * p.N + nb * BN : nullptr;
+      if (valid) p.counts[rec] = static_cast<uint16_t>(cnt);
+      const bool ov = valid && cnt > p.C;
+      if (__any_sync(0xffffffffu, ov)) {
+        int slot = -1;
+        bool fresh = false;
+        if (ov) slot = acquire_row_slot(p.row_slot, p.slot_row, p.r_cap, row, ctrl, fresh);
+        // The lane that opened a slot brings its x row along (whole warp copies).
+        uint32_t fresh_mask = __ballot_sync(0xffffffffu, fresh);
+        while (fresh_mask) {
+          const int src = __ffs(fresh_mask) - 1;
+          fresh_mask &= fresh_mask - 1;
+          const int r = __shfl_sync(0xffffffffu, row, src);
+          const int sl = __shfl_sync(0xffffffffu, slot, src);
+          const uint4* xs = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(r) * p.K);
+          uint4* xd = reinterpret_cast<uint4*>(p.x_over + static_cast<int64_t>(sl) * p.K);
+          for (int v = lane; v < p.K / 8; v += 32) xd[v] = xs[v];
+        }
+        float* dst = slot >= 0 ? p.dense_rows + static_cast<int64_t>(slot) * p.N + t * T : nullptr;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32(taddr + c * 32, r);
-        tmem_wait_ld();
-        if (dst) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+        for (int c = 0; c < T / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32(tcol + c * 32, r);
+          tmem_wait_ld();
+          if (dst) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            d4[v] = make_float4(relu_f(__uint_as_float(r[4 * v + 0])), relu_f(__uint_as_float(r[4 * v + 1])),
-                                relu_f(__uint_as_float(r[4 * v + 2])), relu_f(__uint_as_float(r[4 * v + 3])));
+            for (int v = 0; v < 8; ++v)
+              d4[v] = make_float4(relu_f(__uint_as_float(r[4 * v + 0])), relu_f(__uint_as_float(r[4 * v + 1])),
+                                  relu_f(__uint_as_float(r[4 * v + 2])), relu_f(__uint_as_float(r[4 * v + 3])));
+          }
         }
       }
     }
@@ -174,6 +184,7 @@ struct EpiStoreF32 {
     float* y;
     int ldy;
     int ncols;
+    int accumulate;  // split-K: add into a zero-initialised y with vector atomics
   };
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
@@ -189,13 +200,23 @@ struct EpiStoreF32 {
         float* dst = p.y + static_cast<int64_t>(row) * p.ldy + col0;
         if (col0 + 32 <= p.ncols) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            reinterpret_cast<float4*>(dst)[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          for (int v = 0; v < 8; ++v) {
+            const float4 a = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            if (p.accumulate)
+              atomicAdd(reinterpret_cast<float4*>(dst) + v, a);
+            else
+              reinterpret_cast<float4*>(dst)[v] = a;
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < p.ncols - col0) dst[j] = __uint_as_float(r[j]);
+            if (j < p.ncols - col0) {
+              if (p.accumulate)
+                atomicAdd(dst + j, __uint_as_float(r[j]));
+              else
+                dst[j] = __uint_as_float(r[j]);
+            }
         }
       }
     }
@@ -263,7 +284,8 @@ struct EpiOverflowProduct {
 };
 
 // ---------------------------------------------------------------------------
-// Overflow path, second stage: y[slot_row[r]][col] += acc.
+// Overflow path, second stage: y[slot_row[r]][col] += acc (vector atomics, so
+// split-K slices and the fused kernel's earlier partial sum combine).
 struct EpiAccumulateRows {
   struct Params {
     float* y;
@@ -285,18 +307,14 @@ struct EpiAccumulateRows {
         float* dst = p.y + static_cast<int64_t>(m) * p.ldy + col0;
         if (col0 + 32 <= p.ncols) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            float4 a = reinterpret_cast<float4*>(dst)[v];
-            a.x += __uint_as_float(r[4 * v]);
-            a.y += __uint_as_float(r[4 * v + 1]);
-            a.z += __uint_as_float(r[4 * v + 2]);
-            a.w += __uint_as_float(r[4 * v + 3]);
-            reinterpret_cast<float4*>(dst)[v] = a;
-          }
+          for (int v = 0; v < 8; ++v)
+            atomicAdd(reinterpret_cast<float4*>(dst) + v,
+                      make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                  __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < p.ncols - col0) dst[j] += __uint_as_float(r[j]);
+            if (j < p.ncols - col0) atomicAdd(dst + j, __uint_as_float(r[j]));
         }
       }
     }

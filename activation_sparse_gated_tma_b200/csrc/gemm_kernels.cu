@@ -22,10 +22,11 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap
 
 }  // namespace
 
-cudaError_t launch_gate_twell(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
-                              const EpiGateTwell::Params& p, int* ctrl, int grid, cudaStream_t s) {
-  if (T == 128) return launch<128, false, false, 6, EpiGateTwell>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);
-  if (T == 256) return launch<256, false, false, 4, EpiGateTwell>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);
+cudaError_t launch_gate_twell(int T, int bn, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
+                              const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s) {
+  if (T == 128 && bn == 128) return launch<128, false, false, 6, EpiGateTwell<128>>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);
+  if (T == 128 && bn == 256) return launch<256, false, false, 4, EpiGateTwell<128>>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);
+  if (T == 256 && bn == 256) return launch<256, false, false, 4, EpiGateTwell<256>>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -11,9 +11,10 @@
 
 namespace twell {
 
-// Gate GEMM (tile width T = 128 or 256) with the ReLU + TwELL epilogue.
-cudaError_t launch_gate_twell(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
-                              const EpiGateTwell::Params& p, int* ctrl, int grid, cudaStream_t s);
+// Gate GEMM with the ReLU + TwELL epilogue.  TwELL tile width T in {128, 256};
+// CTA tile width bn in {128, 256}, a multiple of T.
+cudaError_t launch_gate_twell(int T, int bn, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
+                              const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s);
 // h = (x W_u) * ReLU(x W_g), bf16, BN = 128.
 cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
                                  const GemmGeom& g, const EpiGatedProduct::Params& p, int* ctrl, int grid,

@@ -23,7 +23,12 @@ enum : int {
 enum : int {
   kCtrlNOver = 0,      // number of rows that asked for a dense-row slot
   kCtrlFlags = 1,      // status flags
-  kCtrlQueue = 2,      // dynamic token queue of the fused up/down kernel
+  kCtrlQueue = 2,      // fused up/down kernel: next row to take
+  kCtrlDone = 3,       //   warps that finished (the last one rewinds the counters)
+  kCtrlUnitHead = 4,   //   next split-off unit to take
+  kCtrlUnitTail = 5,   //   split-off units published
+  kCtrlScanned = 6,    //   rows whose units are all published
+  kCtrlEpoch = 7,      //   launch epoch (>= 1): tags row flags and unit records
   kCtrlWords = 64,
 };
 

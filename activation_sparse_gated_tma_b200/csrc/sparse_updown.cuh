@@ -3,18 +3,28 @@
 //
 //   y_m = sum_{n in A_m} g_{m,n} * (x_m . W_u[:, n]) * W_d[n, :]
 //
-// Each warp owns one token row at a time; rows come from a dynamic queue so
-// that rows with 10x more active units do not stall a static partition.
-//   * x_m (bf16) and the fp32 accumulator of y_m stay in registers, spread over
-//     the lanes in 16-byte pieces: lane l holds elements [(j*32 + l)*8, +8).
-//   * The warp first lists the row's active units (n, g) from the TwELL
-//     records of its non-overflow tiles into shared memory.
-//   * Lane 0 streams the rows W_u^T[n] and W_d[n] of upcoming list entries
-//     into a private shared-memory ring with 1-D bulk copies (cp.async.bulk,
-//     completion on one mbarrier per slot), several entries ahead, so many
-//     gathers are in flight per SM without holding them in registers.
-//   * For each entry the warp forms u = x_m . W_u^T[n] (warp shuffle reduce),
-//     h = u * g, and accumulates h * W_d[n] into y_m.
+// Work distribution (persistent grid, one CTA per SM, warps independent):
+//   * A warp takes the next token row from a queue.  It scans the row's TwELL
+//     counts; if the row holds more than kUnitCap entries it cuts the row's
+//     tile range into units of about kUnitCap entries, keeps the first unit
+//     and publishes the others on a second queue.  Rows are 100x apart in
+//     active count (the pages report a row maximum above 10x the mean), so a
+//     heavy row is shared by several warps instead of stalling one.
+//   * When the row queue is empty, warps take published units.
+//   * The warp that owns a row (its first unit) stores its partial y_m and
+//     raises the row's flag; warps with later units wait (bounded) for the
+//     flag and add their partial with vector atomics.  The owner was
+//     dequeued before any unit of its row existed, so every wait ends.
+// Inside a unit:
+//   * x_m (bf16) and the fp32 partial of y_m stay in registers, spread over the
+//     lanes in 16-byte pieces: lane l holds elements [(j*32 + l)*8, +8).
+//   * The warp lists the unit's active entries (n, g) from the TwELL records of
+//     its non-overflow tiles into shared memory.
+//   * Lane 0 streams the rows W_u^T[n] and W_d[n] of upcoming entries into a
+//     private shared-memory ring with 1-D bulk copies (cp.async.bulk, no
+//     multicast, one mbarrier per slot), several entries ahead.
+//   * Per entry: u = x_m . W_u^T[n] (warp shuffle reduce), h = u * g,
+//     partial += h * W_d[n].
 // Overflow tiles (count > C) are skipped here; the dense-row path adds them.
 #pragma once
 
@@ -22,7 +32,23 @@
 
 namespace twell {
 
-constexpr int kUpdownListCap = 256;  // list entries per warp and segment
+constexpr int kUpdownListCap = 256;  // list entries per warp and segment (also the N/T limit)
+constexpr int kUnitCap = 64;         // target entries per unit of a split row
+
+struct UpdownParams {
+  const uint16_t* x;
+  const uint16_t* wu_t;
+  const uint16_t* wd;
+  const uint16_t* counts;
+  const uint8_t* idx;
+  const float* vals;
+  int M, K, N, T, C;
+  float* y;
+  int* ctrl;
+  int4* units;     // [M * N/T] published units {row, tile begin, tile end, unused}
+  int* row_flag;   // [M] epoch at which the row's owner stored its partial
+  int stages;
+};
 
 __device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
   const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
@@ -65,6 +91,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -80,149 +116,313 @@ __host__ __device__ constexpr size_t updown_warp_bytes(int K, int stages) {
   return ((static_cast<size_t>(stages) * 4 * K + kUpdownListCap * 8 + stages * 8) + 127) / 128 * 128;
 }
 
+// Per-warp streaming state.
+struct WarpRing {
+  uint8_t* ring;
+  int* list_n;
+  float* list_g;
+  uint64_t* bars;
+  uint32_t slot_bytes;
+  int stages;
+  int head;             // ring slot of the next entry
+  uint32_t head_phase;  // parity that slot's mbarrier completes next
+  uint64_t policy;
+};
+
+// Lists the entries (n, g) of the non-overflow tiles [cursor, te) of `row`
+// into the warp's list, advancing `cursor`; stops before the list would pass
+// its capacity.  Returns the number listed.
+__device__ __forceinline__ int list_entries(const UpdownParams& p, const WarpRing& w, int row, int& cursor, int te,
+                                            int lane) {
+  const int NT = p.N / p.T;
+  const uint16_t* crow = p.counts + static_cast<int64_t>(row) * NT;
+  int E = 0;
+  while (cursor < te) {
+    const int t = cursor + lane;
+    const int c = t < te ? static_cast<int>(crow[t]) : 0;
+    const int ce = (c > 0 && c <= p.C) ? c : 0;
+    const int incl = warp_inclusive_scan(ce, lane);
+    const uint32_t fit = __ballot_sync(0xffffffffu, E + incl <= kUpdownListCap);
+    const int k = __popc(fit);  // fitting lanes form a prefix: incl is non-decreasing
+    if (lane < k && ce > 0) {
+      const int64_t rec = (static_cast<int64_t>(row) * NT + t) * p.C;
+      const int off = E + incl - ce;
+      for (int s = 0; s < ce; ++s) {
+        w.list_n[off + s] = t * p.T + p.idx[rec + s];
+        w.list_g[off + s] = p.vals[rec + s];
+      }
+    }
+    if (k > 0) E += __shfl_sync(0xffffffffu, incl, k - 1);
+    cursor += k;
+    if (k < 32) break;
+  }
+  if (cursor > te) cursor = te;
+  __syncwarp();
+  return E;
+}
+
+__device__ __forceinline__ void issue_entry(const UpdownParams& p, WarpRing& w, int slot, int e) {
+  const int n = w.list_n[e];
+  uint8_t* dst = w.ring + static_cast<size_t>(slot) * w.slot_bytes;
+  mbar_arrive_expect_tx(&w.bars[slot], w.slot_bytes);
+  bulk_load(dst, p.wu_t + static_cast<int64_t>(n) * p.K, w.slot_bytes / 2, &w.bars[slot], w.policy);
+  bulk_load(dst + w.slot_bytes / 2, p.wd + static_cast<int64_t>(n) * p.K, w.slot_bytes / 2, &w.bars[slot], w.policy);
+}
+
+// Streams the E listed entries through the ring and accumulates them.
 template <int KV>
-__global__ void __launch_bounds__(256, 1)
-    twell_updown_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wu_t,
-                        const uint16_t* __restrict__ wd, const uint16_t* __restrict__ counts,
-                        const uint8_t* __restrict__ idx, const float* __restrict__ vals, int M, int K, int N,
-                        int T, int C, float* __restrict__ y, int* ctrl, int stages) {
+__device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& w, int E, const uint4 (&xv)[KV],
+                                               float (&acc)[KV][8], int lane) {
+  const int pre = min(w.stages, E);
+  if (lane == 0) {
+    int s = w.head;
+    for (int e = 0; e < pre; ++e) {
+      issue_entry(p, w, s, e);
+      if (++s == w.stages) s = 0;
+    }
+  }
+  for (int e = 0; e < E; ++e) {
+    const int s = w.head;
+    if (!mbar_wait(&w.bars[s], w.head_phase, p.ctrl)) {
+      // Let the copies still in flight land before the CTA may exit (bounded).
+      int s2 = s;
+      uint32_t ph = w.head_phase;
+      for (int e2 = e; e2 < min(E, e + w.stages); ++e2) {
+        mbar_wait(&w.bars[s2], ph, p.ctrl);
+        if (++s2 == w.stages) { s2 = 0; ph ^= 1u; }
+      }
+      return false;
+    }
+    const uint4* su = reinterpret_cast<const uint4*>(w.ring + static_cast<size_t>(s) * w.slot_bytes);
+    const uint4* sd = su + p.K / 8;  // the W_d row starts 2K bytes into the slot
+    const float g = w.list_g[e];
+    float part = 0.f;
+#pragma unroll
+    for (int j = 0; j < KV; ++j)
+      if ((j * 32 + lane) * 8 < p.K) part += dot8_bf16(xv[j], su[j * 32 + lane]);
+    const float h = warp_sum(part) * g;
+#pragma unroll
+    for (int j = 0; j < KV; ++j)
+      if ((j * 32 + lane) * 8 < p.K) axpy8_bf16(acc[j], h, sd[j * 32 + lane]);
+    __syncwarp();
+    if (lane == 0 && e + w.stages < E) {
+      fence_proxy_async_smem();  // all lanes' reads of slot s precede the refill
+      issue_entry(p, w, s, e + w.stages);
+    }
+    if (++w.head == w.stages) { w.head = 0; w.head_phase ^= 1u; }
+  }
+  return true;
+}
+
+template <int KV>
+__device__ __forceinline__ void load_x(const UpdownParams& p, int row, uint4 (&xv)[KV], float (&acc)[KV][8],
+                                       int lane) {
+  const uint16_t* xr = p.x + static_cast<int64_t>(row) * p.K;
+#pragma unroll
+  for (int j = 0; j < KV; ++j) {
+    const int k0 = (j * 32 + lane) * 8;
+    xv[j] = k0 < p.K ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+  }
+}
+
+template <int KV>
+__device__ __forceinline__ void write_y(const UpdownParams& p, int row, const float (&acc)[KV][8], bool add,
+                                        int lane) {
+  float* yr = p.y + static_cast<int64_t>(row) * p.K;
+#pragma unroll
+  for (int j = 0; j < KV; ++j) {
+    const int k0 = (j * 32 + lane) * 8;
+    if (k0 < p.K) {
+      float4* dst = reinterpret_cast<float4*>(yr + k0);
+      const float4 a = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+      const float4 b = make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+      if (add) {
+        atomicAdd(dst, a);
+        atomicAdd(dst + 1, b);
+      } else {
+        __stcs(dst, a);
+        __stcs(dst + 1, b);
+      }
+    }
+  }
+}
+
+// Unit k of a row covers tiles [cut(k), cut(k+1)); cut(k) is one past the first
+// tile whose inclusive entry prefix reaches ceil(k * total / nunits).
+__device__ __forceinline__ int unit_cut(const int* prefix, int NT, int total, int nunits, int k) {
+  if (k <= 0) return 0;
+  if (k >= nunits) return NT;
+  const int target = static_cast<int>((static_cast<int64_t>(k) * total + nunits - 1) / nunits);
+  int lo = 0, hi = NT - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] >= target)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo + 1;
+}
+
+template <int KV>
+__global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int NT = N / T;
-  const uint32_t slot_bytes = 4u * K;
-  uint8_t* base = smem + static_cast<size_t>(warp) * updown_warp_bytes(K, stages);
-  uint8_t* ring = base;
-  int* list_n = reinterpret_cast<int*>(ring + static_cast<size_t>(stages) * slot_bytes);
-  float* list_g = reinterpret_cast<float*>(list_n + kUpdownListCap);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(list_g + kUpdownListCap);
+  const int NT = p.N / p.T;
+  int* ctrl = p.ctrl;
+
+  WarpRing w;
+  w.slot_bytes = 4u * p.K;
+  w.stages = p.stages;
+  w.ring = smem + static_cast<size_t>(warp) * updown_warp_bytes(p.K, p.stages);
+  w.list_n = reinterpret_cast<int*>(w.ring + static_cast<size_t>(p.stages) * w.slot_bytes);
+  w.list_g = reinterpret_cast<float*>(w.list_n + kUpdownListCap);
+  w.bars = reinterpret_cast<uint64_t*>(w.list_g + kUpdownListCap);
+  w.head = 0;
+  w.head_phase = 0;
   if (lane == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < p.stages; ++s) mbar_init(&w.bars[s], 1);
     fence_barrier_init();
   }
   __syncwarp();
-  const uint64_t policy = l2_evict_last_policy();
+  w.policy = l2_evict_last_policy();
+  const int epoch = ld_acquire(ctrl + kCtrlEpoch);
 
-  int* queue = ctrl + kCtrlQueue;
-  int* done = ctrl + kCtrlQueue + 1;
-  int head = 0;            // ring slot of the next list entry
-  uint32_t head_phase = 0;  // parity that slot's mbarrier completes next
+  uint4 xv[KV];
+  float acc[KV][8];
   bool ok = true;
 
+  // ---------------------------------------------------------------- rows
   while (ok) {
     int row = 0;
-    if (lane == 0) row = atomicAdd(queue, 1);
+    if (lane == 0) row = atomicAdd(ctrl + kCtrlQueue, 1);
     row = __shfl_sync(0xffffffffu, row, 0);
-    if (row >= M) break;
+    if (row >= p.M) break;
+    load_x<KV>(p, row, xv, acc, lane);
 
-    uint4 xv[KV];
-    float acc[KV][8];
-    const uint16_t* xr = x + static_cast<int64_t>(row) * K;
-#pragma unroll
-    for (int j = 0; j < KV; ++j) {
-      const int k0 = (j * 32 + lane) * 8;
-      xv[j] = k0 < K ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+    // Inclusive per-tile prefix of the row's listed entries (list_n as scratch).
+    const uint16_t* crow = p.counts + static_cast<int64_t>(row) * NT;
+    int total = 0;
+    for (int tb = 0; tb < NT; tb += 32) {
+      const int t = tb + lane;
+      const int c = t < NT ? static_cast<int>(crow[t]) : 0;
+      const int ce = (c > 0 && c <= p.C) ? c : 0;
+      const int incl = warp_inclusive_scan(ce, lane);
+      if (t < NT) w.list_n[t] = total + incl;
+      total += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    int nunits = (total + kUnitCap - 1) / kUnitCap;
+    if (nunits > NT) nunits = NT;
+    if (nunits < 1) nunits = 1;
+    const int own_end = unit_cut(w.list_n, NT, total, nunits, 1);
+    if (nunits > 1) {
+      int base = 0;
+      if (lane == 0) base = atomicAdd(ctrl + kCtrlUnitTail, nunits - 1);
+      base = __shfl_sync(0xffffffffu, base, 0);
+      for (int k = 1 + lane; k < nunits; k += 32)
+        p.units[base + k - 1] = make_int4(row, unit_cut(w.list_n, NT, total, nunits, k),
+                                          unit_cut(w.list_n, NT, total, nunits, k + 1), 0);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(ctrl + kCtrlScanned, 1);
     }
 
-    const uint16_t* crow = counts + static_cast<int64_t>(row) * NT;
-    int tile_cursor = 0;
-    while (ok && tile_cursor < NT) {
-      // ---- list the active units of the next tiles (at most kUpdownListCap entries)
-      int E = 0;
-      while (tile_cursor < NT) {
-        const int t = tile_cursor + lane;
-        const int c = t < NT ? static_cast<int>(crow[t]) : 0;
-        const int ce = (c > 0 && c <= C) ? c : 0;
-        const int incl = warp_inclusive_scan(ce, lane);
-        const uint32_t fit = __ballot_sync(0xffffffffu, E + incl <= kUpdownListCap);
-        const int k = __popc(fit);  // fitting lanes form a prefix (incl is non-decreasing)
-        if (lane < k && ce > 0) {
-          const int64_t rec = (static_cast<int64_t>(row) * NT + t) * C;
-          const int off = E + incl - ce;
-          for (int s = 0; s < ce; ++s) {
-            list_n[off + s] = t * T + idx[rec + s];
-            list_g[off + s] = vals[rec + s];
-          }
-        }
-        if (k > 0) E += __shfl_sync(0xffffffffu, incl, k - 1);
-        tile_cursor += min(k, 32);
-        if (k < 32) break;
-      }
-      __syncwarp();
-      if (E == 0) continue;
-
-      // ---- stream the listed rows through the ring
-      const int pre = min(stages, E);
-      if (lane == 0) {
-        int s = head;
-        for (int e = 0; e < pre; ++e) {
-          const int n = list_n[e];
-          uint8_t* dst = ring + static_cast<size_t>(s) * slot_bytes;
-          mbar_arrive_expect_tx(&bars[s], slot_bytes);
-          bulk_load(dst, wu_t + static_cast<int64_t>(n) * K, slot_bytes / 2, &bars[s], policy);
-          bulk_load(dst + slot_bytes / 2, wd + static_cast<int64_t>(n) * K, slot_bytes / 2, &bars[s], policy);
-          if (++s == stages) s = 0;
-        }
-      }
-      int consumed = 0;
-      for (int e = 0; e < E; ++e) {
-        const int s = head;
-        if (!mbar_wait(&bars[s], head_phase, ctrl)) { ok = false; break; }
-        const uint4* su = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(s) * slot_bytes);
-        const uint4* sd = su + K / 8;  // W_d row starts 2K bytes into the slot
-        const float g = list_g[e];
-        float part = 0.f;
-#pragma unroll
-        for (int j = 0; j < KV; ++j)
-          if ((j * 32 + lane) * 8 < K) part += dot8_bf16(xv[j], su[j * 32 + lane]);
-        const float h = warp_sum(part) * g;
-#pragma unroll
-        for (int j = 0; j < KV; ++j)
-          if ((j * 32 + lane) * 8 < K) axpy8_bf16(acc[j], h, sd[j * 32 + lane]);
-        __syncwarp();
-        ++consumed;
-        if (lane == 0 && e + stages < E) {
-          // All lanes finished reading slot s; refill it with entry e + stages.
-          fence_proxy_async_smem();
-          const int n = list_n[e + stages];
-          uint8_t* dst = ring + static_cast<size_t>(s) * slot_bytes;
-          mbar_arrive_expect_tx(&bars[s], slot_bytes);
-          bulk_load(dst, wu_t + static_cast<int64_t>(n) * K, slot_bytes / 2, &bars[s], policy);
-          bulk_load(dst + slot_bytes / 2, wd + static_cast<int64_t>(n) * K, slot_bytes / 2, &bars[s], policy);
-        }
-        if (++head == stages) { head = 0; head_phase ^= 1u; }
-      }
-      if (!ok) {
-        // Let copies already in flight land before the CTA can exit (bounded).
-        int s = head;
-        uint32_t ph = head_phase;
-        for (int e = consumed; e < min(E, consumed + stages); ++e) {
-          mbar_wait(&bars[s], ph, ctrl);
-          if (++s == stages) { s = 0; ph ^= 1u; }
-        }
-      }
-      __syncwarp();
+    int cursor = 0;
+    while (ok && cursor < own_end) {
+      const int E = list_entries(p, w, row, cursor, own_end, lane);
+      if (E > 0) ok = stream_entries<KV>(p, w, E, xv, acc, lane);
     }
     if (!ok) break;
-
-    float* yr = y + static_cast<int64_t>(row) * K;
-#pragma unroll
-    for (int j = 0; j < KV; ++j) {
-      const int k0 = (j * 32 + lane) * 8;
-      if (k0 < K) {
-        __stcs(reinterpret_cast<float4*>(yr + k0), make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]));
-        __stcs(reinterpret_cast<float4*>(yr + k0) + 1, make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]));
-      }
+    write_y<KV>(p, row, acc, false, lane);
+    if (nunits > 1) {
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_release(p.row_flag + row, epoch);
     }
   }
-  // The last warp out rewinds the queue so the next launch starts from row 0.
+
+  // ---------------------------------------------------------------- split-off units
+  // Units are taken only once every row has been scanned, so every reserved
+  // unit record has been written (its writer fenced before counting the row).
+  if (ok) {
+    int ready = 1;
+    if (lane == 0) {
+      const unsigned long long t0 = global_ns();
+      while (ld_acquire(ctrl + kCtrlScanned) < p.M) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          set_flag(ctrl, kFlagWaitTimeout);
+          ready = 0;
+          break;
+        }
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ready, 0) != 0;
+  }
+  const int n_units = ok ? ld_acquire(ctrl + kCtrlUnitTail) : 0;
+  while (ok) {
+    int ux = 0, uy = 0, uz = 0;
+    int have = 0;
+    if (lane == 0) {
+      const int h = atomicAdd(ctrl + kCtrlUnitHead, 1);
+      if (h < n_units) {
+        const int4 u = p.units[h];
+        ux = u.x;
+        uy = u.y;
+        uz = u.z;
+        have = 1;
+      }
+    }
+    have = __shfl_sync(0xffffffffu, have, 0);
+    if (!have) break;
+    const int row = __shfl_sync(0xffffffffu, ux, 0);
+    const int tb = __shfl_sync(0xffffffffu, uy, 0);
+    const int te = __shfl_sync(0xffffffffu, uz, 0);
+    if (tb >= te) continue;
+    load_x<KV>(p, row, xv, acc, lane);
+    int cursor = tb;
+    int listed = 0;
+    while (ok && cursor < te) {
+      const int E = list_entries(p, w, row, cursor, te, lane);
+      listed += E;
+      if (E > 0) ok = stream_entries<KV>(p, w, E, xv, acc, lane);
+    }
+    if (!ok) break;
+    if (listed == 0) continue;
+    // Add after the row's owner has stored its partial (bounded wait).
+    int flag_ok = 1;
+    if (lane == 0) {
+      const unsigned long long t0 = global_ns();
+      while (ld_acquire(p.row_flag + row) != epoch) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          set_flag(ctrl, kFlagWaitTimeout);
+          flag_ok = 0;
+          break;
+        }
+      }
+    }
+    flag_ok = __shfl_sync(0xffffffffu, flag_ok, 0);
+    if (!flag_ok) break;
+    write_y<KV>(p, row, acc, true, lane);
+  }
+
+  // The last warp out rewinds the queues and opens the next epoch.
   if (lane == 0) {
+    __threadfence();
     const int total = gridDim.x * (blockDim.x >> 5);
-    if (atomicAdd(done, 1) == total - 1) {
-      atomicExch(queue, 0);
-      atomicExch(done, 0);
+    if (atomicAdd(ctrl + kCtrlDone, 1) == total - 1) {
+      ctrl[kCtrlQueue] = 0;
+      ctrl[kCtrlUnitHead] = 0;
+      ctrl[kCtrlUnitTail] = 0;
+      ctrl[kCtrlScanned] = 0;
+      ctrl[kCtrlEpoch] = epoch + 1;
+      __threadfence();
+      ctrl[kCtrlDone] = 0;
     }
   }
 }

@@ -33,6 +33,7 @@ struct GemmGeom {
   const int* m_limit;       // optional: only rows < min(M, *m_limit) are computed
   int group_m;              // rasterisation: tiles walk group_m row blocks per column sweep
   int b_k_wrap;             // if > 0, B's k-block index is kb % b_k_wrap (A = [A0 | A1] against B twice)
+  int k_splits;             // >= 1: the reduction is cut into k_splits slices, each its own tile
 };
 
 template <int BN, bool DUAL>
@@ -84,8 +85,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (g.m_limit) m_rows = min(m_rows, *g.m_limit);
   const int num_m = (m_rows + kBM - 1) / kBM;
   const int num_n = (g.N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
-  const int num_kb = g.K / kBK;
+  const int num_mn = num_m * num_n;
+  const int k_splits = g.k_splits > 1 ? g.k_splits : 1;
+  const int num_tiles = num_mn * k_splits;
+  const int total_kb = g.K / kBK;
+  const int kb_per_split = (total_kb + k_splits - 1) / k_splits;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -116,9 +120,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         int mb, nb;
-        tile_coords(tile, num_m, num_n, g.group_m, mb, nb);
+        tile_coords(tile % num_mn, num_m, num_n, g.group_m, mb, nb);
+        const int kb0 = (tile / num_mn) * kb_per_split;
+        const int kb1 = min(total_kb, kb0 + kb_per_split);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, ctrl)) { ok = false; break; }
           uint8_t* sa = smem + stage * L::kStageBytes;
           uint8_t* sb = sa + L::kABytes;
@@ -152,8 +158,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, ctrl)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * L::kAccCols;
+        const int kb0 = (tile / num_mn) * kb_per_split;
+        const int kb1 = min(total_kb, kb0 + kb_per_split);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, ctrl)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + stage * L::kStageBytes);
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t adesc = smem_desc_sw128(a_base + k * 32, 16, 1024);
             const uint64_t bdesc = B_MN ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
                                         : smem_desc_sw128(b_base + k * 32, 16, 1024);
-            const uint32_t accum = (kb | k) != 0;
+            const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
             umma_bf16(d, adesc, bdesc, idesc, accum);
             if (DUAL) {
               const uint32_t b2 = b_base + L::kBBytes;
@@ -185,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       int mb, nb;
-      tile_coords(tile, num_m, num_n, g.group_m, mb, nb);
+      tile_coords(tile % num_mn, num_m, num_n, g.group_m, mb, nb);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       if (!mbar_wait(&tfull[acc], acc_phase, ctrl)) break;

@@ -20,6 +20,30 @@ namespace {
 thread_local char g_err[512] = "";
 thread_local int g_launches = 0;
 
+// Optional launch tracing: events[2i] / events[2i+1] bracket the i-th kernel.
+struct Trace {
+  cudaEvent_t* events = nullptr;
+  int capacity = 0;
+  int count = 0;
+  const char* names[256];
+};
+thread_local Trace g_trace;
+
+cudaError_t trace_begin(cudaStream_t s) {
+  if (g_trace.events && g_trace.count < g_trace.capacity) return cudaEventRecord(g_trace.events[2 * g_trace.count], s);
+  return cudaSuccess;
+}
+cudaError_t trace_end(cudaStream_t s, const char* name) {
+  ++g_launches;
+  if (g_trace.events && g_trace.count < g_trace.capacity) {
+    cudaError_t e = cudaEventRecord(g_trace.events[2 * g_trace.count + 1], s);
+    if (e != cudaSuccess) return e;
+    if (g_trace.count < 256) g_trace.names[g_trace.count] = name;
+    ++g_trace.count;
+  }
+  return cudaSuccess;
+}
+
 twell_status fail(twell_status st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -111,11 +135,12 @@ twell_status tmap_bf16(const void* ptr, uint64_t inner, uint64_t outer, uint32_t
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, total;
+  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, units, row_flag, total;
 };
 
 bool shape_ok(int M, int K, int N, int T, int C, int R_cap) {
   return M >= 1 && K >= 64 && K <= 4096 && K % 64 == 0 && (T == 128 || T == 256) && N >= T && N % T == 0 &&
+         N / T <= kUpdownListCap &&
          C >= 1 && C <= T && C <= 255 && R_cap >= 1 && static_cast<int64_t>(M) * N < (int64_t(1) << 40);
 }
 
@@ -132,6 +157,8 @@ Layout layout(int M, int K, int N, int T, int C, int R_cap) {
   L.dense_rows = o; o = align256(o + size_t(R_cap) * N * 4);
   L.x_over = o; o = align256(o + size_t(R_cap) * K * 2);
   L.h_over = o; o = align256(o + size_t(R_cap) * N * 4);
+  L.units = o; o = align256(o + size_t(M) * NT * 16);
+  L.row_flag = o; o = align256(o + size_t(M) * 4);
   L.total = o;
   return L;
 }
@@ -140,17 +167,22 @@ twell_status check_buf(const twell_buf* tw) {
   if (!tw) return fail(TWELL_ERR_INVALID, "twell_buf is NULL");
   if (!shape_ok(tw->M, tw->K, tw->N, tw->T, tw->C, tw->R_cap)) return fail(TWELL_ERR_INVALID, "twell_buf has invalid sizes");
   if (!tw->counts || !tw->idx || !tw->vals || !tw->dense_rows || !tw->row_slot || !tw->slot_row || !tw->ctrl ||
-      !tw->x_over || !tw->h_over)
+      !tw->x_over || !tw->h_over || !tw->units || !tw->row_flag)
     return fail(TWELL_ERR_INVALID, "twell_buf is not initialised");
   return TWELL_OK;
 }
 
 // ---------------------------------------------------------------- small kernels
 // Start of a gate pass: no row holds a dense-row slot, control words at zero.
-__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl) {
+// The fused kernel's epoch starts at 1 so that zeroed row flags mean "not stored".
+__global__ void twell_reset_kernel(int* __restrict__ row_slot, int* __restrict__ row_flag, int M,
+                                   int* __restrict__ ctrl) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < kCtrlWords) ctrl[i] = 0;
-  for (int r = i; r < M; r += gridDim.x * blockDim.x) row_slot[r] = kSlotFree;
+  if (i < kCtrlWords) ctrl[i] = (i == kCtrlEpoch) ? 1 : 0;
+  for (int r = i; r < M; r += gridDim.x * blockDim.x) {
+    row_slot[r] = kSlotFree;
+    row_flag[r] = 0;
+  }
 }
 
 // Warps per CTA and ring depth of the fused kernel for a given K: eight warps
@@ -177,12 +209,13 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
   cudaError_t e = cudaFuncSetAttribute(twell_updown_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int rows_per_wave = warps;
-  int grid = sms;
-  const int max_grid = (tw->M + rows_per_wave - 1) / rows_per_wave;
-  if (grid > max_grid) grid = max_grid;
-  twell_updown_kernel<KV><<<grid, 32 * warps, smem, s>>>(x, wu_t, wd, tw->counts, tw->idx, tw->vals, tw->M, tw->K,
-                                                        tw->N, tw->T, tw->C, y, tw->ctrl, stages);
+  UpdownParams p;
+  p.x = x; p.wu_t = wu_t; p.wd = wd;
+  p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals;
+  p.M = tw->M; p.K = tw->K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
+  p.y = y; p.ctrl = tw->ctrl; p.units = reinterpret_cast<int4*>(tw->units); p.row_flag = tw->row_flag;
+  p.stages = stages;
+  twell_updown_kernel<KV><<<sms, 32 * warps, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -200,9 +233,21 @@ cudaError_t launch_updown(const uint16_t* x, const uint16_t* wu_t, const uint16_
   }
 }
 
-int gemm_grid(int rows, int cols, int bn, int sms) {
-  const long tiles = static_cast<long>((rows + kBM - 1) / kBM) * ((cols + bn - 1) / bn);
+int gemm_grid(int rows, int cols, int bn, int sms, int k_splits = 1) {
+  const long tiles = static_cast<long>((rows + kBM - 1) / kBM) * ((cols + bn - 1) / bn) * k_splits;
   return static_cast<int>(tiles < sms ? tiles : sms);
+}
+
+// Reduction slices for a GEMM with few output tiles: enough tiles to cover the
+// SMs, every slice at least 8 k-blocks long and none empty.
+int choose_k_splits(int rows, int cols, int bn, int K, int sms) {
+  const int tiles = ((rows + kBM - 1) / kBM) * ((cols + bn - 1) / bn);
+  const int kb = K / kBK;
+  int splits = (sms + tiles - 1) / tiles;
+  if (splits > kb / 8) splits = kb / 8;
+  if (splits < 1) return 1;
+  const int per = (kb + splits - 1) / splits;
+  return (kb + per - 1) / per;
 }
 
 }  // namespace
@@ -228,6 +273,20 @@ const char* twell_last_error(void) { return g_err; }
 
 int twell_last_launch_count(void) { return g_launches; }
 
+twell_status twell_trace_events(cudaEvent_t* events, int capacity) {
+  if (events && capacity < 1) return fail(TWELL_ERR_INVALID, "capacity must be >= 1");
+  g_trace.events = events;
+  g_trace.capacity = events ? capacity : 0;
+  g_trace.count = 0;
+  return TWELL_OK;
+}
+
+int twell_trace_count(void) { return g_trace.count; }
+
+const char* twell_trace_name(int i) {
+  return (i >= 0 && i < g_trace.count && i < 256) ? g_trace.names[i] : nullptr;
+}
+
 size_t twell_buf_bytes(int M, int K, int N, int T, int C, int R_cap) {
   if (!shape_ok(M, K, N, T, C, R_cap)) return 0;
   return layout(M, K, N, T, C, R_cap).total;
@@ -251,6 +310,8 @@ twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int 
   tw->dense_rows = reinterpret_cast<float*>(b + L.dense_rows);
   tw->x_over = reinterpret_cast<uint16_t*>(b + L.x_over);
   tw->h_over = reinterpret_cast<uint16_t*>(b + L.h_over);
+  tw->units = b + L.units;
+  tw->row_flag = reinterpret_cast<int32_t*>(b + L.row_flag);
   tw->M = M; tw->K = K; tw->N = N; tw->T = T; tw->C = C; tw->R_cap = R_cap;
   return TWELL_OK;
 }
@@ -266,22 +327,27 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
   DeviceInfo dev;
   if ((st = device_info(dev)) != TWELL_OK) return st;
 
+  // 256-wide CTA tiles halve the operand traffic per FLOP; 128-wide ones give
+  // small-M problems twice the CTAs.
+  const int bn = (N % 256 == 0 && (M > 256 || tw->T == 256)) ? 256 : 128;
   CUtensorMap tm_x, tm_wg;
   if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(wg_t, K, N, tw->T, tm_wg)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wg_t, K, N, bn, tm_wg)) != TWELL_OK) return st;
 
   const int rgrid = static_cast<int>((static_cast<int64_t>(M) + 255) / 256 < 1024 ? (M + 255) / 256 : 1024);
-  twell_reset_kernel<<<rgrid > 0 ? rgrid : 1, 256, 0, stream>>>(tw->row_slot, M, tw->ctrl);
+  TW_CUDA(trace_begin(stream));
+  twell_reset_kernel<<<rgrid > 0 ? rgrid : 1, 256, 0, stream>>>(tw->row_slot, tw->row_flag, M, tw->ctrl);
   TW_CUDA(cudaGetLastError());
-  ++g_launches;
+  TW_CUDA(trace_end(stream, "twell_reset"));
 
-  EpiGateTwell::Params p;
+  GateTwellParams p;
   p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.dense_rows = tw->dense_rows;
   p.row_slot = tw->row_slot; p.slot_row = tw->slot_row; p.x = x; p.x_over = tw->x_over;
   p.N = N; p.K = K; p.C = tw->C; p.r_cap = tw->R_cap;
-  GemmGeom g{M, N, K, nullptr, kGateGroupM, 0};
-  TW_CUDA(launch_gate_twell(tw->T, tm_x, tm_wg, g, p, tw->ctrl, gemm_grid(M, N, tw->T, dev.sms), stream));
-  ++g_launches;
+  GemmGeom g{M, N, K, nullptr, kGateGroupM, 0, 1};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_gate_twell(tw->T, bn, tm_x, tm_wg, g, p, tw->ctrl, gemm_grid(M, N, bn, dev.sms), stream));
+  TW_CUDA(trace_end(stream, "gate_twell_gemm"));
 
   if (n_over_host) {
     int n_over = 0;
@@ -321,8 +387,9 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
   if ((st = device_info(dev)) != TWELL_OK) return st;
   const int N = tw->N;
 
+  TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_updown(x, wu_t, wd, tw, y, dev.sms, stream));
-  ++g_launches;
+  TW_CUDA(trace_end(stream, "twell_updown"));
 
   // Dense-row path for overflow tiles; rows beyond the device-side n_over are skipped.
   CUtensorMap tm_xo, tm_wu, tm_ho, tm_wd;
@@ -334,15 +401,18 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
   EpiOverflowProduct::Params p1;
   p1.counts = tw->counts; p1.dense_rows = tw->dense_rows; p1.slot_row = tw->slot_row; p1.h_over = tw->h_over;
   p1.N = N; p1.T = tw->T; p1.C = tw->C;
-  GemmGeom g1{tw->R_cap, N, K, tw->ctrl + kCtrlNOver, kGateGroupM, 0};
+  GemmGeom g1{tw->R_cap, N, K, tw->ctrl + kCtrlNOver, kGateGroupM, 0, 1};
+  TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_overflow_product(tm_xo, tm_wu, g1, p1, tw->ctrl, gemm_grid(tw->R_cap, N, 128, dev.sms), stream));
-  ++g_launches;
+  TW_CUDA(trace_end(stream, "overflow_up_gemm"));
 
   EpiAccumulateRows::Params p2;
   p2.y = y; p2.slot_row = tw->slot_row; p2.ldy = K; p2.ncols = K;
-  GemmGeom g2{tw->R_cap, K, 2 * N, tw->ctrl + kCtrlNOver, kGateGroupM, N / kBK};
-  TW_CUDA(launch_overflow_down(tm_ho, tm_wd, g2, p2, tw->ctrl, gemm_grid(tw->R_cap, K, 256, dev.sms), stream));
-  ++g_launches;
+  const int ks2 = choose_k_splits(tw->R_cap, K, 256, 2 * N, dev.sms);
+  GemmGeom g2{tw->R_cap, K, 2 * N, tw->ctrl + kCtrlNOver, kGateGroupM, N / kBK, ks2};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_overflow_down(tm_ho, tm_wd, g2, p2, tw->ctrl, gemm_grid(tw->R_cap, K, 256, dev.sms, ks2), stream));
+  TW_CUDA(trace_end(stream, "overflow_down_gemm"));
   return TWELL_OK;
 }
 
@@ -364,13 +434,17 @@ twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   if ((st = tmap_bf16(wd, K, N, 64, tm_wd)) != TWELL_OK) return st;
 
   EpiGatedProduct::Params p1{h_scratch, N};
-  GemmGeom g1{M, N, K, nullptr, kGateGroupM, 0};
+  GemmGeom g1{M, N, K, nullptr, kGateGroupM, 0, 1};
+  TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_gated_product(tm_x, tm_wg, tm_wu, g1, p1, nullptr, gemm_grid(M, N, 128, dev.sms), stream));
-  ++g_launches;
-  EpiStoreF32::Params p2{y, K, K};
-  GemmGeom g2{M, K, N, nullptr, kGateGroupM, 0};
-  TW_CUDA(launch_down_store(tm_h, tm_wd, g2, p2, nullptr, gemm_grid(M, K, 256, dev.sms), stream));
-  ++g_launches;
+  TW_CUDA(trace_end(stream, "dense_gate_up_gemm"));
+  const int ks2 = choose_k_splits(M, K, 256, N, dev.sms);
+  if (ks2 > 1) TW_CUDA(cudaMemsetAsync(y, 0, static_cast<size_t>(M) * K * sizeof(float), stream));
+  EpiStoreF32::Params p2{y, K, K, ks2 > 1 ? 1 : 0};
+  GemmGeom g2{M, K, N, nullptr, kGateGroupM, 0, ks2};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_down_store(tm_h, tm_wd, g2, p2, nullptr, gemm_grid(M, K, 256, dev.sms, ks2), stream));
+  TW_CUDA(trace_end(stream, "dense_down_gemm"));
   return TWELL_OK;
 }
 

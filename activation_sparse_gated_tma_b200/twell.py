@@ -36,7 +36,8 @@ class CapacityError(TwellError):
 
 class _TwellBuf(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("counts", "idx", "vals", "dense_rows", "row_slot", "slot_row", "ctrl", "x_over", "h_over")] + \
+                ("counts", "idx", "vals", "dense_rows", "row_slot", "slot_row", "ctrl", "x_over", "h_over",
+                 "units", "row_flag")] + \
                [(n, ctypes.c_int) for n in ("M", "K", "N", "T", "C", "R_cap")]
 
 
@@ -66,6 +67,9 @@ def lib() -> ctypes.CDLL:
         "twell_status_str": (ctypes.c_char_p, [I]),
         "twell_last_error": (ctypes.c_char_p, []),
         "twell_last_launch_count": (I, []),
+        "twell_trace_events": (I, [P, I]),
+        "twell_trace_count": (I, []),
+        "twell_trace_name": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -90,6 +94,39 @@ def _check(status: int, where: str):
 
 def last_launch_count() -> int:
     return lib().twell_last_launch_count()
+
+
+class KernelTrace:
+    """Brackets every kernel the library launches (on this thread) with CUDA
+    events, for per-kernel device times of live runs.
+
+        with KernelTrace(capacity=16) as tr:
+            ...library calls...
+        torch.cuda.synchronize(); tr.times_ms() -> [(kernel name, ms), ...]
+    """
+
+    def __init__(self, capacity: int = 16):
+        self.capacity = capacity
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.events:      # torch creates the CUDA event lazily, on first record
+            e.record()
+        self._arr = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.events])
+        self.count = 0
+        self.names = []
+
+    def __enter__(self):
+        _check(lib().twell_trace_events(self._arr, self.capacity), "twell_trace_events")
+        return self
+
+    def __exit__(self, *exc):
+        L = lib()
+        self.count = L.twell_trace_count()
+        self.names = [L.twell_trace_name(i).decode() for i in range(self.count)]
+        L.twell_trace_events(None, 0)
+        return False
+
+    def times_ms(self):
+        return [(self.names[i], self.events[2 * i].elapsed_time(self.events[2 * i + 1])) for i in range(self.count)]
 
 
 def _stream(stream=None) -> int:

@@ -1,0 +1,445 @@
+"""Throughput of the sparse gated FFN forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+One step = one pass of the whole sparse path over one batch of M tokens:
+twell_gate_pack (reset + tcgen05 gate GEMM with the ReLU/TwELL/overflow
+epilogue) followed by twell_ffn_fwd (fused sparse up+down kernel, then the
+dense-row overflow GEMMs), asynchronous, inputs resident in HBM.  The L2
+(126 MB) is flushed with a 256 MiB write before every timed step; the flush
+is outside the timed events.
+
+For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
+same workload: the forward pass is token-parallel and needs no collective
+("replicas only", weak scaling); times are the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the test oracle, unchanged) on the
+host cores for the same workload and metric, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from activation_sparse_gated_tma_b200 import workloads as wl  # noqa: E402
+
+METRIC = "sparse FFN fwd tokens/s @99% sparsity, % of roofline, speedup vs own dense FFN"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILES = os.path.join(ROOT, "profiles")
+FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; a profile taken on other sources is stale."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "activation_sparse_gated_tma_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from a committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(PROFILES, f"{kernel}__{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7], "sw_power": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def workload_stats(tw, w, T, C):
+    counts = tw.counts.cpu().numpy().view(np.uint16).astype(np.int64)
+    per_tok = counts.sum(1)
+    ov = counts > C
+    return {
+        "active_fraction": float(per_tok.sum() / (w.M * w.N)),
+        "nnz_per_token_mean": float(per_tok.mean()),
+        "nnz_per_token_p50": float(np.percentile(per_tok, 50)),
+        "nnz_per_token_p99": float(np.percentile(per_tok, 99)),
+        "nnz_per_token_max": int(per_tok.max()),
+        "overflow_rows": int(ov.any(1).sum()),
+        "overflow_tiles": int(ov.sum()),
+        "twell_entries": int(np.where(ov, 0, counts).sum()),
+    }
+
+
+def unique_active_units(tw, C, T):
+    """Number of distinct hidden units read by the fused kernel (non-overflow entries)."""
+    counts = tw.counts.cpu().numpy().view(np.uint16).astype(np.int64)
+    idx = tw.idx.cpu().numpy().astype(np.int64)
+    M, NT = counts.shape
+    used = (np.arange(C)[None, None, :] < np.minimum(counts, C)[:, :, None]) & (counts <= C)[:, :, None]
+    t_i = np.broadcast_to(np.arange(NT)[None, :, None], idx.shape)
+    n = (t_i * T + idx)[used]
+    return int(np.unique(n).size)
+
+
+def cpu_oracle_rate(d, w, rows_target_s: float, min_rows: int = 8):
+    """Time the fp64 oracle's sparse forward (gate, TwELL pack, sparse y) on a
+    bounded row sample; returns (tokens/s, rows, seconds, threads)."""
+    import oracle
+    nthreads = oracle.default_threads()
+    probe = wl.subsample_rows(w.M, max(min_rows, nthreads), seed=5)
+    t0 = time.perf_counter()
+    oracle.forward(d["x"], d["wg_t"], d["wu_t"], d["wd"], w.T, w.C, rows=probe, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    per_row = dt / probe.size
+    n = int(max(min_rows, min(w.M, rows_target_s / max(per_row, 1e-9))))
+    n = max(nthreads, (n // nthreads) * nthreads) if n >= nthreads else n
+    rows = wl.subsample_rows(w.M, n, seed=6)
+    t0 = time.perf_counter()
+    oracle.forward(d["x"], d["wg_t"], d["wu_t"], d["wd"], w.T, w.C, rows=rows, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return rows.size / dt, int(rows.size), dt, nthreads
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    d = wl.generate(w)
+    import oracle
+    nthreads = oracle.default_threads()
+    # Size one step to about 2 s of CPU work so --steps K --warmup W ends in minutes.
+    probe = wl.subsample_rows(w.M, max(8, nthreads), seed=5)
+    t0 = time.perf_counter()
+    oracle.forward(d["x"], d["wg_t"], d["wu_t"], d["wd"], w.T, w.C, rows=probe, nthreads=nthreads)
+    per_row = (time.perf_counter() - t0) / probe.size
+    rows_per_step = int(min(w.M, max(nthreads, 2.0 / max(per_row, 1e-9))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = wl.subsample_rows(w.M, rows_per_step, seed=100 + i)
+        t0 = time.perf_counter()
+        oracle.forward(d["x"], d["wg_t"], d["wu_t"], d["wd"], w.T, w.C, rows=rows, nthreads=nthreads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = rows_per_step / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "T": w.T, "C": w.C,
+                   "rows_per_step": rows_per_step},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": f"{rows_per_step} seeded rows of {w.M} per step: fp64 gate, TwELL pack, sparse y"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- native arm
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from activation_sparse_gated_tma_b200 import twell as tw
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = wl.WORKLOADS[args.workload]
+    d = wl.generate(w)
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, wg, wu, wd = (to_dev(d[k]) for k in ("x", "wg_t", "wu_t", "wd"))
+    M, K, N, T, C = w.M, w.K, w.N, w.T, w.C
+    tb = tw.TwellBuffers(M, K, N, T, C, device=dev)
+    y = torch.empty(M, K, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        tw.gate_pack(x, wg, tb)
+        n1 = tw.last_launch_count()
+        tw.ffn_fwd(x, wu, wd, tb, y)
+        return n1 + tw.last_launch_count()
+
+    # Correctness of the configuration before timing: capacity and device flags.
+    step()
+    st, n_over, flags = tw.read_status(tb)
+    if st != tw.OK:
+        raise RuntimeError(f"sparse path status {st} (n_over={n_over}, flags={flags}); raise R_cap")
+    stats = workload_stats(tb, w, T, C)
+    U = unique_active_units(tb, C, T)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    traces = []
+    launches = 0
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            tr = tw.KernelTrace(capacity=8)
+            with tr:
+                starts[i].record()
+                launches += step()
+                ends[i].record()
+            traces.append(tr)
+        torch.cuda.synchronize()
+        barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+    per_kernel = {}
+    for tr in traces:
+        for name, t in tr.times_ms():
+            per_kernel.setdefault(name, []).append(t)
+    kern_ms = {k: sum(v) / len(v) for k, v in per_kernel.items()}
+
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # In-build dense tcgen05 FFN on the same inputs (same flush discipline).
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        tw.dense_ffn(x, wg, wu, wd, h, y)
+    dense_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        tw.dense_ffn(x, wg, wu, wd, h, y)
+        b.record()
+        b.synchronize()
+        dense_ms.append(a.elapsed_time(b))
+    dense_ms = sum(dense_ms) / len(dense_ms)
+    if world > 1:
+        t = torch.tensor([dense_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dense_ms = float(t.item())
+
+    # End to end through the public API with host buffers: pinned x in, y out.
+    x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty(M, K, dtype=torch.float32).pin_memory()
+    x_e2e = torch.empty_like(x)
+
+    def e2e_step():
+        x_e2e.copy_(x_host, non_blocking=True)
+        tw.gate_pack(x_e2e, wg, tb)
+        tw.ffn_fwd(x_e2e, wu, wd, tb, y)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    e2e_ms = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        e2e_step()
+        b.record()
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_ms = sum(e2e_ms) / len(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        return
+
+    peaks, peak_kind = load_peaks()
+    # Algorithmic quantities per launch / per step.
+    flops_gate = 2.0 * M * K * N
+    NT = N // T
+    bytes_updown = (2.0 * M * K                      # x rows
+                    + 2.0 * M * NT                   # counts
+                    + 5.0 * stats["twell_entries"]   # idx + fp32 value per listed entry
+                    + 4.0 * K * U                    # unique W_u^T and W_d rows
+                    + 4.0 * M * K)                   # y (fp32)
+    R = n_over
+    flops_over = 2.0 * R * K * N * 2                 # up and down GEMMs of the slotted rows
+    bytes_path = (2.0 * K * N + 4.0 * K * U + 2.0 * M * K + 4.0 * M * K + 2.0 * M * NT * (2 + 5 * C)
+                  + 8.0 * R * N)
+    t_roof_s = max((flops_gate + flops_over) / (peaks["bf16_tflops"] * 1e12), bytes_path / (peaks["hbm_gbs"] * 1e9))
+    kernels = {}
+    for name, t in kern_ms.items():
+        if name == "gate_twell_gemm":
+            ach = flops_gate / (t * 1e-3) / 1e12
+            kernels[name] = {"ms": t, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
+        elif name == "twell_updown":
+            ach = bytes_updown / (t * 1e-3) / 1e9
+            kernels[name] = {"ms": t, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": ach / peaks["hbm_gbs"],
+                             "l2_gather_gbs": 4.0 * K * stats["twell_entries"] / (t * 1e-3) / 1e9}
+        else:
+            kernels[name] = {"ms": t}
+    dominant = max(kern_ms.items(), key=lambda kv: kv[1])[0]
+    dom = kernels[dominant]
+    roofline = {"kernel": dominant, "bound": dom.get("bound"), "achieved": dom.get("achieved"),
+                "peak": dom.get("peak"), "unit": dom.get("unit"), "frac": dom.get("frac"),
+                "traffic": profiled_traffic(dominant, w.name), "peak_source": peak_kind + " (burst)"}
+
+    cpu = None
+    if not args.no_cpu_baseline:
+        rate, rows, sec, cores = cpu_oracle_rate(d, w, rows_target_s=12.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{rows} seeded rows of {w.M} ({sec:.1f} s): fp64 gate, TwELL pack, sparse y"}
+
+    value = world * M / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "C": C, "R_cap": w.R_cap,
+                   "global_batch": world * M, "parallelism": f"replicas{world}",
+                   "l2": "flushed: 256 MiB write before each timed step (outside the timed events)",
+                   "mode": "asynchronous gate_pack (overflow count stays on the device)"},
+        "sparsity": stats, "unique_units_gathered": U,
+        "roofline": roofline,
+        "path_roofline": {"t_roof_ms": t_roof_s * 1e3, "frac": t_roof_s * 1e3 / ms,
+                          "bound": "tensor" if (flops_gate + flops_over) / (peaks["bf16_tflops"] * 1e12)
+                          >= bytes_path / (peaks["hbm_gbs"] * 1e9) else "hbm",
+                          "flops": flops_gate + flops_over, "bytes": bytes_path},
+        "kernels": kernels,
+        "dense": {"ms_per_step": dense_ms, "value": world * M / (dense_ms * 1e-3), "unit": UNIT},
+        "speedup_vs_dense": dense_ms / ms,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * M / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 2 * M * K,
+                "d2h_bytes_per_step": 4 * M * K, "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=wl.BENCH_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -74,6 +74,8 @@ typedef enum {
  *   x_over     bf16   [R_cap][K]  scratch: gathered x rows of slotted rows
  *   h_over     bf16   [R_cap][2N] scratch: overflow-tile hidden activations as
  *                                 bf16 hi (columns < N) + lo (columns >= N) parts
+ *   units      int32  [M*NT][4]   scratch: work units of rows split across warps
+ *   row_flag   int32  [M]         scratch: per-row publication flags of the fused kernel
  */
 typedef struct twell_buf {
   uint16_t* counts;
@@ -85,6 +87,8 @@ typedef struct twell_buf {
   int32_t* ctrl;
   uint16_t* x_over;
   uint16_t* h_over;
+  void* units;
+  int32_t* row_flag;
   int M, K, N, T, C, R_cap;
 } twell_buf;
 
@@ -95,8 +99,8 @@ size_t twell_buf_bytes(int M, int K, int N, int T, int C, int R_cap);
  * Carve `base` (device pointer, >= twell_buf_bytes(...) bytes, 256-byte
  * aligned) into the arrays of `tw`.  Host-side pointer arithmetic only; the
  * contents are initialised by twell_gate_pack.  Limits: M >= 1, K % 64 == 0,
- * 64 <= K <= 4096, T in {128, 256}, N % T == 0, 1 <= C <= min(T, 255),
- * 1 <= R_cap.
+ * 64 <= K <= 4096, T in {128, 256}, N % T == 0, N / T <= 256,
+ * 1 <= C <= min(T, 255), 1 <= R_cap.
  */
 twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int K, int N, int T, int C,
                             int R_cap);
@@ -153,6 +157,19 @@ const char* twell_last_error(void);
 
 /* Number of kernels the last call on this thread enqueued (for launch accounting). */
 int twell_last_launch_count(void);
+
+/*
+ * Per-kernel timing hook.  After twell_trace_events(events, capacity) with an
+ * array of 2*capacity caller-created CUDA events, each kernel that later
+ * calls on this thread enqueue is bracketed by cudaEventRecord(events[2i]) and
+ * cudaEventRecord(events[2i+1]) on the call's stream, for the first `capacity`
+ * kernels.  twell_trace_count() returns how many were recorded and
+ * twell_trace_name(i) the kernel's name (static string).  Passing NULL turns
+ * tracing off.  Tracing adds event records only; the work is unchanged.
+ */
+twell_status twell_trace_events(cudaEvent_t* events, int capacity);
+int twell_trace_count(void);
+const char* twell_trace_name(int i);
 
 #ifdef __cplusplus
 }

@@ -32,6 +32,7 @@ def test_status_strings():
     (64, 256, 1024, 128, 0, 1),     # C < 1
     (64, 256, 1024, 128, 129, 1),   # C > T
     (64, 256, 1024, 128, 8, 0),     # R_cap < 1
+    (64, 256, 128 * 257, 128, 8, 1),  # N / T > 256
 ])
 def test_buf_bytes_rejects_invalid_sizes(args):
     assert tw.lib().twell_buf_bytes(*args) == 0
@@ -46,9 +47,9 @@ def test_buf_init_layout_is_aligned_and_disjoint():
     b = tw._TwellBuf()
     assert L.twell_buf_init(ctypes.byref(b), base, nbytes, M, K, N, T, C, R) == tw.OK
     NT = N // T
-    spans = [("ctrl", 64 * 4), ("counts", M * NT * 2), ("idx", M * NT * C), ("vals", M * NT * C * 2),
-             ("row_slot", M * 4), ("slot_row", R * 4), ("dense_rows", R * N * 2), ("x_over", R * K * 2),
-             ("h_over", R * N * 2)]
+    spans = [("ctrl", 64 * 4), ("counts", M * NT * 2), ("idx", M * NT * C), ("vals", M * NT * C * 4),
+             ("row_slot", M * 4), ("slot_row", R * 4), ("dense_rows", R * N * 4), ("x_over", R * K * 2),
+             ("h_over", R * N * 4), ("units", M * NT * 16), ("row_flag", M * 4)]
     ranges = []
     for name, size in spans:
         p = getattr(b, name)
