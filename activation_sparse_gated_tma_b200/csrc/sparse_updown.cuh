@@ -33,7 +33,7 @@
 namespace twell {
 
 constexpr int kUpdownListCap = 256;  // list entries per warp and segment (also the N/T limit)
-constexpr int kUnitCap = 64;         // target entries per unit of a split row
+constexpr int kUnitCap = 16;         // target entries per unit of a split row
 
 struct UpdownParams {
   const uint16_t* x;
@@ -85,10 +85,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
           smem_u32(smem_dst)),
       "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -204,11 +200,8 @@ __device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& 
 #pragma unroll
     for (int j = 0; j < KV; ++j)
       if ((j * 32 + lane) * 8 < p.K) axpy8_bf16(acc[j], h, sd[j * 32 + lane]);
-    __syncwarp();
-    if (lane == 0 && e + w.stages < E) {
-      fence_proxy_async_smem();  // all lanes' reads of slot s precede the refill
-      issue_entry(p, w, s, e + w.stages);
-    }
+    __syncwarp();  // every lane's reads of slot s are done before lane 0 refills it
+    if (lane == 0 && e + w.stages < E) issue_entry(p, w, s, e + w.stages);
     if (++w.head == w.stages) { w.head = 0; w.head_phase ^= 1u; }
   }
   return true;

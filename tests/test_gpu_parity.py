@@ -155,8 +155,8 @@ def test_repeat_calls_are_deterministic():
     # produced by one warp alone: bit-identical.  Rows split across warps and
     # slotted rows add partials with fp32 atomics, whose order varies.
     listed = np.where(h1["counts"] <= C, h1["counts"], 0).astype(np.int64).sum(1)
-    plain = torch.from_numpy((h1["row_slot"] < 0) & (listed <= 64)).cuda()
-    assert int(plain.sum()) > w.M // 2
+    plain = torch.from_numpy((h1["row_slot"] < 0) & (listed <= 8)).cuda()
+    assert int(plain.sum()) > w.M // 4
     assert torch.equal(y1[plain], y2[plain])
     torch.testing.assert_close(y1[~plain], y2[~plain], rtol=1e-5, atol=1e-5 * float(y1.abs().max()))
     # the fused kernel reuses its work queue across launches
