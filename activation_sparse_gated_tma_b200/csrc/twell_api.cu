@@ -449,3 +449,52 @@ twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Dense FFN for callers that cannot allocate device memory at call time: a
+// runtime that has handed all device memory to its own pool, or an embedding
+// that forbids allocation while it executes.  The hidden activations h, which
+// dense_ffn_fwd takes as a caller buffer, live here in a fixed array that is
+// part of the library's device image; every device that loads the library
+// keeps it (32 MiB) until the process exits.
+namespace twell {
+namespace {
+
+constexpr size_t kNoAllocHiddenElems = size_t(16) << 20;  // 16 Mi bf16 values = 32 MiB
+__device__ __align__(256) uint16_t g_noalloc_hidden[kNoAllocHiddenElems];
+
+// Device address of the fixed array on the current device.  In host code the
+// array's name is only a host-side handle, so the address is looked up once per
+// device (with that device current) and cached.
+twell_status noalloc_hidden_ptr(uint16_t** out) {
+  int dev = 0;
+  TW_CUDA(cudaGetDevice(&dev));
+  static std::mutex mu;
+  static std::map<int, uint16_t*> addr;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = addr.find(dev);
+  if (it == addr.end()) {
+    void* p = nullptr;
+    TW_CUDA(cudaGetSymbolAddress(&p, g_noalloc_hidden));
+    it = addr.emplace(dev, static_cast<uint16_t*>(p)).first;
+  }
+  *out = it->second;
+  return TWELL_OK;
+}
+
+}  // namespace
+}  // namespace twell
+
+extern "C" twell_status dense_ffn_fwd_noalloc(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t,
+                                              const uint16_t* wd, int M, int K, int N, float* y,
+                                              cudaStream_t stream) {
+  g_launches = 0;
+  if (M < 1 || N < 1 || static_cast<size_t>(M) * static_cast<size_t>(N) > kNoAllocHiddenElems)
+    return fail(TWELL_ERR_INVALID,
+                "dense_ffn_fwd_noalloc: M*N = %lld exceeds the built-in scratch of %zu elements (32 MiB of bf16)",
+                static_cast<long long>(M) * N, kNoAllocHiddenElems);
+  uint16_t* h = nullptr;
+  twell_status st = noalloc_hidden_ptr(&h);
+  if (st != TWELL_OK) return st;
+  return dense_ffn_fwd(x, wg_t, wu_t, wd, M, K, N, h, y, stream);
+}

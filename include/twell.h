@@ -149,6 +149,27 @@ twell_status twell_read_status(const twell_buf* tw, int* n_over_host, int* devic
 twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
                            int M, int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream);
 
+/*
+ * dense_ffn_fwd without a caller-provided hidden buffer, for callers that
+ * cannot allocate device memory when they call (a runtime that has handed all
+ * device memory to its own pool, or an embedding that forbids allocation while
+ * it executes).  The pages describe no such variant; it is an interface
+ * convenience of this library.
+ *
+ * The hidden activations use a fixed 32 MiB array inside the library's device
+ * image (every device that loads the library holds it until the process exits),
+ * so M * N must not exceed 16,777,216; larger problems return
+ * TWELL_ERR_INVALID with a message and launch nothing.  No device memory is
+ * allocated or freed by this call.  The first call on a device looks up the
+ * array's device address (with that device current); make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents, so calls that overlap on the GPU (other streams, other
+ * host threads) race on it; serialise them.  Otherwise identical to
+ * dense_ffn_fwd: y [M][K] fp32 is overwritten, asynchronous on `stream`.
+ */
+twell_status dense_ffn_fwd_noalloc(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
+                                   int M, int K, int N, float* y, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char* twell_status_str(twell_status status);
 
