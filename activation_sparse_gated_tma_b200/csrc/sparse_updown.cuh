@@ -165,7 +165,21 @@ __device__ __forceinline__ void issue_entry(const UpdownParams& p, WarpRing& w, 
   bulk_load(dst + w.slot_bytes / 2, p.wd + static_cast<int64_t>(n) * p.K, w.slot_bytes / 2, &w.bars[slot], w.policy);
 }
 
-// Streams the E listed entries through the ring and accumulates them.
+__device__ __forceinline__ float dot8_acc(const uint4& a, const uint4& b, float s) {
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+  const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    s = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), s);
+    s = fmaf(__uint_as_float(aw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), s);
+  }
+  return s;
+}
+
+// Streams the E listed entries through the ring and accumulates them.  Entries
+// are taken two at a time: the two dot products, their shuffle reductions and
+// the two accumulations are independent, so each warp keeps twice the work in
+// flight per dependency chain.
 template <int KV>
 __device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& w, int E, const uint4 (&xv)[KV],
                                                float (&acc)[KV][8], int lane) {
@@ -177,32 +191,58 @@ __device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& 
       if (++s == w.stages) s = 0;
     }
   }
-  for (int e = 0; e < E; ++e) {
-    const int s = w.head;
-    if (!mbar_wait(&w.bars[s], w.head_phase, p.ctrl)) {
+  auto slot = [&](int s) { return reinterpret_cast<const uint4*>(w.ring + static_cast<size_t>(s) * w.slot_bytes); };
+  for (int e = 0; e < E; e += 2) {
+    const bool two = e + 1 < E;
+    const int sa = w.head;
+    const uint32_t pa = w.head_phase;
+    const int sb = sa + 1 == w.stages ? 0 : sa + 1;
+    const uint32_t pb = sa + 1 == w.stages ? (pa ^ 1u) : pa;
+    bool ok = mbar_wait(&w.bars[sa], pa, p.ctrl);
+    if (ok && two) ok = mbar_wait(&w.bars[sb], pb, p.ctrl);
+    if (!ok) {
       // Let the copies still in flight land before the CTA may exit (bounded).
-      int s2 = s;
-      uint32_t ph = w.head_phase;
+      int s2 = sa;
+      uint32_t ph = pa;
       for (int e2 = e; e2 < min(E, e + w.stages); ++e2) {
         mbar_wait(&w.bars[s2], ph, p.ctrl);
         if (++s2 == w.stages) { s2 = 0; ph ^= 1u; }
       }
       return false;
     }
-    const uint4* su = reinterpret_cast<const uint4*>(w.ring + static_cast<size_t>(s) * w.slot_bytes);
-    const uint4* sd = su + p.K / 8;  // the W_d row starts 2K bytes into the slot
-    const float g = w.list_g[e];
-    float part = 0.f;
+    const uint4* ua = slot(sa);
+    const uint4* ub = slot(sb);
+    float part_a = 0.f, part_b = 0.f;
 #pragma unroll
-    for (int j = 0; j < KV; ++j)
-      if ((j * 32 + lane) * 8 < p.K) part += dot8_bf16(xv[j], su[j * 32 + lane]);
-    const float h = warp_sum(part) * g;
+    for (int j = 0; j < KV; ++j) {
+      if ((j * 32 + lane) * 8 < p.K) {
+        part_a = dot8_acc(xv[j], ua[j * 32 + lane], part_a);
+        if (two) part_b = dot8_acc(xv[j], ub[j * 32 + lane], part_b);
+      }
+    }
 #pragma unroll
-    for (int j = 0; j < KV; ++j)
-      if ((j * 32 + lane) * 8 < p.K) axpy8_bf16(acc[j], h, sd[j * 32 + lane]);
-    __syncwarp();  // every lane's reads of slot s are done before lane 0 refills it
-    if (lane == 0 && e + w.stages < E) issue_entry(p, w, s, e + w.stages);
-    if (++w.head == w.stages) { w.head = 0; w.head_phase ^= 1u; }
+    for (int o = 16; o > 0; o >>= 1) {
+      part_a += __shfl_xor_sync(0xffffffffu, part_a, o);
+      part_b += __shfl_xor_sync(0xffffffffu, part_b, o);
+    }
+    const float ha = part_a * w.list_g[e];
+    const float hb = two ? part_b * w.list_g[e + 1] : 0.f;
+    const uint4* da = ua + p.K / 8;  // the W_d row starts 2K bytes into the slot
+    const uint4* db = ub + p.K / 8;
+#pragma unroll
+    for (int j = 0; j < KV; ++j) {
+      if ((j * 32 + lane) * 8 < p.K) {
+        axpy8_bf16(acc[j], ha, da[j * 32 + lane]);
+        if (two) axpy8_bf16(acc[j], hb, db[j * 32 + lane]);
+      }
+    }
+    __syncwarp();  // every lane's reads of the two slots are done before they are refilled
+    // Lanes 0 and 1 refill the two slots in one instruction.
+    const int refill = e + (lane & 1) + w.stages;
+    if (lane < (two ? 2 : 1) && refill < E) issue_entry(p, w, lane == 0 ? sa : sb, refill);
+    const int used = two ? 2 : 1;
+    w.head += used;
+    if (w.head >= w.stages) { w.head -= w.stages; w.head_phase ^= 1u; }
   }
   return true;
 }
