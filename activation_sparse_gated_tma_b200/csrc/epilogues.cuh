@@ -48,6 +48,15 @@ __device__ __forceinline__ int acquire_row_slot(int* row_slot, int* slot_row, in
 
 __device__ __forceinline__ float relu_f(float z) { return z > 0.f ? z : 0.f; }
 
+// Epilogue interface (see tc_gemm.cuh): Pre<BN> holds what prepare() loads
+// before the accumulator is ready; run() consumes it.  Most epilogues need none.
+struct EpiNoPrepare {
+  template <int BN>
+  struct Pre {};
+  template <int BN, class Params>
+  static __device__ __forceinline__ void prepare(const Params&, Pre<BN>&, int, int, int) {}
+};
+
 // ---------------------------------------------------------------------------
 // Gate epilogue: ReLU + TwELL packing + overflow routing ("Sparser, Faster,
 // Lighter Transformer Language Models", §3-4 steps 3-5 and §3-6).
@@ -67,13 +76,18 @@ struct GateTwellParams {
 };
 
 template <int T>
-struct EpiGateTwell {
+struct EpiGateTwell : EpiNoPrepare {
   using Params = GateTwellParams;
+  // Per epilogue warp: one 32-column chunk of its 32 rows, laid out
+  // [column][lane] so that every thread's dynamically indexed reads of its own
+  // row hit distinct banks.
+  static constexpr int kScratchBytes = 32 * 32 * 4;
 
   template <int BN>
-  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb,
-                                             int lane, int* ctrl) {
+  static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
+                                             int nb, int lane, int* ctrl, void* scratch) {
     static_assert(BN % T == 0, "a CTA tile must hold whole TwELL tiles");
+    float* stage = static_cast<float*>(scratch) + lane;
     const bool valid = row < m_rows;
     const int NT = p.N / T;
 #pragma unroll 1
@@ -89,19 +103,24 @@ struct EpiGateTwell {
         uint32_t r[32];
         tmem_ld_32x32(tcol + c * 32, r);
         tmem_wait_ld();
-        if (valid) {
+        // Bit j: column c*32+j is active (ReLU(z) > 0).
+        uint32_t mask = 0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float z = __uint_as_float(r[j]);
-            if (z > 0.f) {
-              if (cnt < p.C) {
-                idx_rec[cnt] = static_cast<uint8_t>(c * 32 + j);
-                val_rec[cnt] = z;
-              }
-              ++cnt;
-            }
+        for (int j = 0; j < 32; ++j) mask |= (__uint_as_float(r[j]) > 0.f ? 1u : 0u) << j;
+        if (!valid) mask = 0;
+        if (mask != 0 && cnt < p.C) {
+          // Stage the chunk, then pack only the set bits, in ascending column order.
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stage[j * 32] = __uint_as_float(r[j]);
+          while (mask != 0 && cnt < p.C) {
+            const int j = __ffs(mask) - 1;
+            mask &= mask - 1;
+            idx_rec[cnt] = static_cast<uint8_t>(c * 32 + j);
+            val_rec[cnt] = stage[j * 32];
+            ++cnt;
           }
         }
+        cnt += __popc(mask);
       }
       if (valid) p.counts[rec] = static_cast<uint16_t>(cnt);
       const bool ov = valid && cnt > p.C;
@@ -143,14 +162,15 @@ struct EpiGateTwell {
 // Dense FFN first stage: accumulator 0 = x W_g tile, accumulator 1 = x W_u
 // tile (same columns).  Writes h = h_u * ReLU(h_g) as bf16 ("Sparser, Faster,
 // Lighter Transformer Language Models", §1-1).
-struct EpiGatedProduct {
+struct EpiGatedProduct : EpiNoPrepare {
+  static constexpr int kScratchBytes = 0;
   struct Params {
     uint16_t* h;  // [M][N] bf16
     int N;
   };
   template <int BN>
-  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
-                                             int*) {
+  static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
+                                             int nb, int, int*, void*) {
     const bool valid = row < m_rows;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
@@ -179,7 +199,8 @@ struct EpiGatedProduct {
 
 // ---------------------------------------------------------------------------
 // Plain fp32 store of the accumulator: y[row][col] = acc, col < ncols.
-struct EpiStoreF32 {
+struct EpiStoreF32 : EpiNoPrepare {
+  static constexpr int kScratchBytes = 0;
   struct Params {
     float* y;
     int ldy;
@@ -187,8 +208,8 @@ struct EpiStoreF32 {
     int accumulate;  // split-K: add into a zero-initialised y with vector atomics
   };
   template <int BN>
-  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
-                                             int*) {
+  static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
+                                             int nb, int, int*, void*) {
     const bool valid = row < m_rows;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
@@ -231,6 +252,7 @@ struct EpiStoreF32 {
 // unevaluated sum of two bf16 numbers (hi + lo, |lo| <= 2^-9 |hi|) so that the
 // second stage keeps ~16 bits of h while feeding bf16 tensor cores.
 struct EpiOverflowProduct {
+  static constexpr int kScratchBytes = 0;
   struct Params {
     const uint16_t* counts;   // [M][N/T]
     const float* dense_rows;  // [R_cap][N]
@@ -239,35 +261,45 @@ struct EpiOverflowProduct {
     int N, T, C;
   };
   template <int BN>
-  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
-                                             int*) {
-    const bool valid = row < m_rows;
-    const int m = valid ? p.slot_row[row] : -1;
+  struct Pre {
+    float g[BN];  // the row's stored ReLU gate on the tile's columns (overflow tiles only)
+    bool ov;      // the row's TwELL tile under these columns overflowed
+  };
+  template <int BN>
+  static __device__ __forceinline__ void prepare(const Params& p, Pre<BN>& pre, int row, int m_rows, int nb) {
+    const int m = row < m_rows ? p.slot_row[row] : -1;
     const int NT = p.N / p.T;
     const int t = (nb * BN) / p.T;
-    const bool ov = m >= 0 && p.counts[static_cast<int64_t>(m) * NT + t] > p.C;
-#pragma unroll 1
+    pre.ov = m >= 0 && p.counts[static_cast<int64_t>(m) * NT + t] > p.C;
+    if (pre.ov) {
+      const float4* src = reinterpret_cast<const float4*>(p.dense_rows + static_cast<int64_t>(row) * p.N + nb * BN);
+#pragma unroll
+      for (int v = 0; v < BN / 4; ++v) {
+        const float4 a = src[v];
+        pre.g[4 * v + 0] = a.x;
+        pre.g[4 * v + 1] = a.y;
+        pre.g[4 * v + 2] = a.z;
+        pre.g[4 * v + 3] = a.w;
+      }
+    }
+  }
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, const Pre<BN>& pre, uint32_t taddr, int row, int m_rows,
+                                             int nb, int, int*, void*) {
+    const bool valid = row < m_rows;
+#pragma unroll
     for (int c = 0; c < BN / 32; ++c) {
       uint32_t u[32];
       tmem_ld_32x32(taddr + c * 32, u);
       tmem_wait_ld();
       if (valid) {
-        const int64_t off = static_cast<int64_t>(row) * p.N + nb * BN + c * 32;
         uint4* dst_hi = reinterpret_cast<uint4*>(p.h_over + static_cast<int64_t>(row) * 2 * p.N + nb * BN + c * 32);
         uint4* dst_lo = dst_hi + p.N / 8;
-        const float4* gsrc = reinterpret_cast<const float4*>(p.dense_rows + off);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           float h[8];
-          if (ov) {
-            const float4 g0 = gsrc[2 * v], g1 = gsrc[2 * v + 1];
-            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) h[e] = __uint_as_float(u[8 * v + e]) * g[e];
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) h[e] = 0.f;
-          }
+          for (int e = 0; e < 8; ++e) h[e] = pre.ov ? __uint_as_float(u[8 * v + e]) * pre.g[c * 32 + 8 * v + e] : 0.f;
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -286,7 +318,8 @@ struct EpiOverflowProduct {
 // ---------------------------------------------------------------------------
 // Overflow path, second stage: y[slot_row[r]][col] += acc (vector atomics, so
 // split-K slices and the fused kernel's earlier partial sum combine).
-struct EpiAccumulateRows {
+struct EpiAccumulateRows : EpiNoPrepare {
+  static constexpr int kScratchBytes = 0;
   struct Params {
     float* y;
     const int* slot_row;
@@ -294,8 +327,8 @@ struct EpiAccumulateRows {
     int ncols;
   };
   template <int BN>
-  static __device__ __forceinline__ void run(const Params& p, uint32_t taddr, int row, int m_rows, int nb, int,
-                                             int*) {
+  static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
+                                             int nb, int, int*, void*) {
     const int m = row < m_rows ? p.slot_row[row] : -1;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {

@@ -9,15 +9,14 @@ namespace {
 template <int BN, bool B_MN, bool DUAL, int STAGES, class Epi>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmGeom& g,
                    const typename Epi::Params& ep, int* ctrl, int grid, cudaStream_t s) {
-  constexpr size_t smem = gemm_smem_bytes<BN, DUAL, STAGES>();
+  constexpr size_t smem = gemm_smem_bytes<BN, DUAL, STAGES, Epi::kScratchBytes>();
   static_assert(smem <= 232448, "exceeds the 227 KB per-CTA shared memory limit");
   auto kern = tc_gemm_kernel<BN, B_MN, DUAL, STAGES, Epi>;
   // The attribute is per device; setting it is cheap and idempotent.
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kGemmThreads, smem, s>>>(a, b, b2, g, ep, ctrl);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, kGemmThreads, smem, s, a, b, b2, g, ep, ctrl);
 }
 
 }  // namespace
@@ -41,9 +40,11 @@ cudaError_t launch_down_store(const CUtensorMap& tm_h, const CUtensorMap& tm_wd,
   return launch<256, true, false, 4, EpiStoreF32>(tm_h, tm_wd, tm_wd, g, p, ctrl, grid, s);
 }
 
-cudaError_t launch_overflow_product(const CUtensorMap& tm_xo, const CUtensorMap& tm_wu, const GemmGeom& g,
+cudaError_t launch_overflow_product(int bn, const CUtensorMap& tm_xo, const CUtensorMap& tm_wu, const GemmGeom& g,
                                     const EpiOverflowProduct::Params& p, int* ctrl, int grid, cudaStream_t s) {
-  return launch<128, false, false, 6, EpiOverflowProduct>(tm_xo, tm_wu, tm_wu, g, p, ctrl, grid, s);
+  if (bn == 64) return launch<64, false, false, 8, EpiOverflowProduct>(tm_xo, tm_wu, tm_wu, g, p, ctrl, grid, s);
+  if (bn == 128) return launch<128, false, false, 6, EpiOverflowProduct>(tm_xo, tm_wu, tm_wu, g, p, ctrl, grid, s);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_overflow_down(const CUtensorMap& tm_ho, const CUtensorMap& tm_wd, const GemmGeom& g,

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "epilogues.cuh"
 #include "tc_gemm.cuh"
 
@@ -22,13 +24,32 @@ cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_
 // y = h W_d (W_d stored [N][K], read MN-major), fp32 store, BN = 256.
 cudaError_t launch_down_store(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const GemmGeom& g,
                               const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s);
-// Overflow rows: h_over = (x_over W_u) * dense_rows on overflow tiles, BN = 128.
-cudaError_t launch_overflow_product(const CUtensorMap& tm_xo, const CUtensorMap& tm_wu, const GemmGeom& g,
+// Overflow rows: h_over = (x_over W_u) * dense_rows on overflow tiles, BN in {64, 128}.
+cudaError_t launch_overflow_product(int bn, const CUtensorMap& tm_xo, const CUtensorMap& tm_wu, const GemmGeom& g,
                                     const EpiOverflowProduct::Params& p, int* ctrl, int grid, cudaStream_t s);
 // Overflow rows: y[slot_row[r]] += h_over[r] W_d, BN = 256.
 cudaError_t launch_overflow_down(const CUtensorMap& tm_ho, const CUtensorMap& tm_wd, const GemmGeom& g,
                                  const EpiAccumulateRows::Params& p, int* ctrl, int grid, cudaStream_t s);
 
 constexpr int kGateGroupM = 16;
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel in the stream is still running.  Every kernel of
+// this library issues griddepcontrol.wait before its first global memory
+// access, so ordering is kept; only the launch and set-up overlap.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace twell

@@ -49,6 +49,15 @@ __device__ __forceinline__ void set_flag(int* ctrl, int flag) {
   if (ctrl) atomicOr(ctrl + kCtrlFlags, flag);
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: the next kernel in the stream may be scheduled
+// once every CTA of this one has signalled (or exited); it must wait for this
+// grid's completion before reading what this grid wrote.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -50,24 +50,21 @@ struct UpdownParams {
   int stages;
 };
 
-__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
-  const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-  const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
-  float s = 0.f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    s = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), s);
-    s = fmaf(__uint_as_float(aw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), s);
-  }
-  return s;
-}
-
+// acc += h * d for 8 bf16 elements of d, as four packed fp32x2 FMAs (each lane
+// of a pair rounds exactly as a scalar fp32 FMA would).
 __device__ __forceinline__ void axpy8_bf16(float (&acc)[8], float h, const uint4& d) {
   const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    acc[2 * e] = fmaf(h, __uint_as_float(dw[e] << 16), acc[2 * e]);
-    acc[2 * e + 1] = fmaf(h, __uint_as_float(dw[e] & 0xFFFF0000u), acc[2 * e + 1]);
+    const float lo = __uint_as_float(dw[e] << 16);
+    const float hi = __uint_as_float(dw[e] & 0xFFFF0000u);
+    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+        "mov.b64 pa, {%2, %3};\n\t"
+        "mov.b64 pb, {%4, %4};\n\t"
+        "mov.b64 pc, {%0, %1};\n\t"
+        "fma.rn.f32x2 pc, pa, pb, pc;\n\t"
+        "mov.b64 {%0, %1}, pc;\n\t}"
+        : "+f"(acc[2 * e]), "+f"(acc[2 * e + 1]) : "f"(lo), "f"(hi), "f"(h));
   }
 }
 
@@ -165,21 +162,29 @@ __device__ __forceinline__ void issue_entry(const UpdownParams& p, WarpRing& w, 
   bulk_load(dst + w.slot_bytes / 2, p.wd + static_cast<int64_t>(n) * p.K, w.slot_bytes / 2, &w.bars[slot], w.policy);
 }
 
-__device__ __forceinline__ float dot8_acc(const uint4& a, const uint4& b, float s) {
+// s[e] += the products of the e-th bf16 pair of a and b: four independent
+// accumulation chains per entry instead of one.  The mixed-precision FMA takes
+// the bf16 halves as they are (the product of two bf16 numbers is exact in
+// fp32), so no unpacking is needed; the result equals fp32 FMAs on the
+// widened values.
+__device__ __forceinline__ void dot8_acc4(const uint4& a, const uint4& b, float (&s)[4]) {
   const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
   const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    s = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), s);
-    s = fmaf(__uint_as_float(aw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), s);
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "+f"(s[e]) : "r"(aw[e]), "r"(bw[e]));
   }
-  return s;
 }
 
 // Streams the E listed entries through the ring and accumulates them.  Entries
-// are taken two at a time: the two dot products, their shuffle reductions and
-// the two accumulations are independent, so each warp keeps twice the work in
-// flight per dependency chain.
+// are taken two at a time: the two dot products (four partial sums each), their
+// shuffle reductions and the two accumulations are independent, so each warp
+// keeps several short dependency chains in flight instead of one long one.
 template <int KV>
 __device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& w, int E, const uint4 (&xv)[KV],
                                                float (&acc)[KV][8], int lane) {
@@ -212,14 +217,16 @@ __device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& 
     }
     const uint4* ua = slot(sa);
     const uint4* ub = slot(sb);
-    float part_a = 0.f, part_b = 0.f;
+    float qa[4] = {0.f, 0.f, 0.f, 0.f}, qb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < KV; ++j) {
       if ((j * 32 + lane) * 8 < p.K) {
-        part_a = dot8_acc(xv[j], ua[j * 32 + lane], part_a);
-        if (two) part_b = dot8_acc(xv[j], ub[j * 32 + lane], part_b);
+        dot8_acc4(xv[j], ua[j * 32 + lane], qa);
+        if (two) dot8_acc4(xv[j], ub[j * 32 + lane], qb);
       }
     }
+    float part_a = (qa[0] + qa[1]) + (qa[2] + qa[3]);
+    float part_b = (qb[0] + qb[1]) + (qb[2] + qb[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       part_a += __shfl_xor_sync(0xffffffffu, part_a, o);
@@ -322,6 +329,9 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
   }
   __syncwarp();
   w.policy = l2_evict_last_policy();
+  // Set-up above overlaps the previous kernel (programmatic dependent launch).
+  griddep_launch_dependents();
+  griddep_wait();
   const int epoch = ld_acquire(ctrl + kCtrlEpoch);
 
   uint4 xv[KV];

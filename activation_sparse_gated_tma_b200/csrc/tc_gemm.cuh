@@ -10,7 +10,8 @@
 //   warp 0      TMA producer (one elected lane) filling a STAGES-deep smem ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //   warps 2..5  epilogue: thread i of warp w owns TMEM lane 32*(w%4)+i, i.e.
-//               one output row of the 128-row tile, and runs Epi::run on it.
+//               one output row of the 128-row tile; per tile it runs
+//               Epi::prepare (before the accumulator is ready) and Epi::run.
 // Accumulators are double-buffered in TMEM so the epilogue of tile i overlaps
 // the MMAs of tile i+1.  Every wait is bounded (see mbar_wait).
 #pragma once
@@ -33,7 +34,9 @@ struct GemmGeom {
   const int* m_limit;       // optional: only rows < min(M, *m_limit) are computed
   int group_m;              // rasterisation: tiles walk group_m row blocks per column sweep
   int b_k_wrap;             // if > 0, B's k-block index is kb % b_k_wrap (A = [A0 | A1] against B twice)
-  int k_splits;             // >= 1: the reduction is cut into k_splits slices, each its own tile
+  int k_splits;             // >= 1: the reduction is cut into k_splits slices, each its own tile;
+                            // < 0: as many slices (at most -k_splits) as keep the live tiles
+                            // (rows below *m_limit) within one pass of the grid
 };
 
 template <int BN, bool DUAL>
@@ -47,10 +50,12 @@ struct GemmSmem {
   static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte swizzle-atom alignment");
 };
 
-template <int BN, bool DUAL, int STAGES>
+// Shared memory of one CTA: the operand ring, the barriers, and EPI_SCRATCH
+// bytes of private scratch for each of the four epilogue warps.
+template <int BN, bool DUAL, int STAGES, int EPI_SCRATCH>
 constexpr size_t gemm_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * GemmSmem<BN, DUAL>::kStageBytes +
-         (2 * STAGES + 4) * sizeof(uint64_t) + 16;
+         (2 * STAGES + 4) * sizeof(uint64_t) + 16 + 128 + 4 * static_cast<size_t>(EPI_SCRATCH);
 }
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int& mb, int& nb) {
@@ -77,19 +82,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint8_t* epi_scratch = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tmem_holder + 4) + 127) & ~uintptr_t(127));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  int m_rows = g.M;
-  if (g.m_limit) m_rows = min(m_rows, *g.m_limit);
-  const int num_m = (m_rows + kBM - 1) / kBM;
-  const int num_n = (g.N + BN - 1) / BN;
-  const int num_mn = num_m * num_n;
-  const int k_splits = g.k_splits > 1 ? g.k_splits : 1;
-  const int num_tiles = num_mn * k_splits;
-  const int total_kb = g.K / kBK;
-  const int kb_per_split = (total_kb + k_splits - 1) / k_splits;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -110,6 +106,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+
+  // Everything above overlaps the tail of the previous kernel in the stream
+  // (programmatic dependent launch); global memory is touched only below.
+  griddep_launch_dependents();
+  griddep_wait();
+
+  int m_rows = g.M;
+  if (g.m_limit) m_rows = min(m_rows, *g.m_limit);
+  const int num_m = (m_rows + kBM - 1) / kBM;
+  const int num_n = (g.N + BN - 1) / BN;
+  const int num_mn = num_m * num_n;
+  const int total_kb = g.K / kBK;
+  int k_splits = g.k_splits > 1 ? g.k_splits : 1;
+  if (g.k_splits < 0) {
+    k_splits = num_mn > 0 ? static_cast<int>(gridDim.x) / num_mn : 1;
+    k_splits = max(1, min(k_splits, -g.k_splits));
+  }
+  const int kb_per_split = (total_kb + k_splits - 1) / k_splits;
+  k_splits = (total_kb + kb_per_split - 1) / kb_per_split;  // no empty slice
+  const int num_tiles = num_mn * k_splits;
 
   if (warp == 0) {
     if (lane == 0 && num_tiles > blockIdx.x) {
@@ -196,11 +212,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tile_coords(tile % num_mn, num_m, num_n, g.group_m, mb, nb);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      // Loads that do not depend on the accumulator are issued while the MMAs run.
+      typename Epi::template Pre<BN> pre;
+      Epi::template prepare<BN>(ep, pre, mb * kBM + row_in_tile, m_rows, nb);
       if (!mbar_wait(&tfull[acc], acc_phase, ctrl)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
-      Epi::template run<BN>(ep, taddr, mb * kBM + row_in_tile, m_rows, nb, lane, ctrl);
+      Epi::template run<BN>(ep, pre, taddr, mb * kBM + row_in_tile, m_rows, nb, lane, ctrl,
+                            epi_scratch + (warp - 2) * Epi::kScratchBytes);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

@@ -177,6 +177,8 @@ twell_status check_buf(const twell_buf* tw) {
 // The fused kernel's epoch starts at 1 so that zeroed row flags mean "not stored".
 __global__ void twell_reset_kernel(int* __restrict__ row_slot, int* __restrict__ row_flag, int M,
                                    int* __restrict__ ctrl) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < kCtrlWords) ctrl[i] = (i == kCtrlEpoch) ? 1 : 0;
   for (int r = i; r < M; r += gridDim.x * blockDim.x) {
@@ -215,8 +217,7 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
   p.M = tw->M; p.K = tw->K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
   p.y = y; p.ctrl = tw->ctrl; p.units = reinterpret_cast<int4*>(tw->units); p.row_flag = tw->row_flag;
   p.stages = stages;
-  twell_updown_kernel<KV><<<sms, 32 * warps, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(twell_updown_kernel<KV>, sms, 32 * warps, smem, s, p);
 }
 
 cudaError_t launch_updown(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw, float* y,
@@ -238,12 +239,13 @@ int gemm_grid(int rows, int cols, int bn, int sms, int k_splits = 1) {
   return static_cast<int>(tiles < sms ? tiles : sms);
 }
 
-// Reduction slices for a GEMM with few output tiles: enough tiles to cover the
-// SMs, every slice at least 8 k-blocks long and none empty.
+// Reduction slices for a GEMM with few output tiles: as many as keep all
+// tiles in one wave on the SMs, every slice at least 8 k-blocks long and none
+// empty.
 int choose_k_splits(int rows, int cols, int bn, int K, int sms) {
   const int tiles = ((rows + kBM - 1) / kBM) * ((cols + bn - 1) / bn);
   const int kb = K / kBK;
-  int splits = (sms + tiles - 1) / tiles;
+  int splits = sms / tiles;
   if (splits > kb / 8) splits = kb / 8;
   if (splits < 1) return 1;
   const int per = (kb + splits - 1) / splits;
@@ -336,8 +338,8 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
 
   const int rgrid = static_cast<int>((static_cast<int64_t>(M) + 255) / 256 < 1024 ? (M + 255) / 256 : 1024);
   TW_CUDA(trace_begin(stream));
-  twell_reset_kernel<<<rgrid > 0 ? rgrid : 1, 256, 0, stream>>>(tw->row_slot, tw->row_flag, M, tw->ctrl);
-  TW_CUDA(cudaGetLastError());
+  TW_CUDA(launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, stream, tw->row_slot, tw->row_flag, M,
+                     tw->ctrl));
   TW_CUDA(trace_end(stream, "twell_reset"));
 
   GateTwellParams p;
@@ -394,7 +396,9 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
   // Dense-row path for overflow tiles; rows beyond the device-side n_over are skipped.
   CUtensorMap tm_xo, tm_wu, tm_ho, tm_wd;
   if ((st = tmap_bf16(tw->x_over, K, tw->R_cap, kBM, tm_xo)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(wu_t, K, N, 128, tm_wu)) != TWELL_OK) return st;
+  // Narrow tiles when the slotted rows are too few to occupy the SMs with 128-wide ones.
+  const int bn1 = static_cast<long>((tw->R_cap + kBM - 1) / kBM) * (N / 128) * 2 <= dev.sms ? 64 : 128;
+  if ((st = tmap_bf16(wu_t, K, N, bn1, tm_wu)) != TWELL_OK) return st;
   if ((st = tmap_bf16(tw->h_over, 2 * N, tw->R_cap, kBM, tm_ho)) != TWELL_OK) return st;
   if ((st = tmap_bf16(wd, K, N, 64, tm_wd)) != TWELL_OK) return st;
 
@@ -403,15 +407,18 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
   p1.N = N; p1.T = tw->T; p1.C = tw->C;
   GemmGeom g1{tw->R_cap, N, K, tw->ctrl + kCtrlNOver, kGateGroupM, 0, 1};
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_overflow_product(tm_xo, tm_wu, g1, p1, tw->ctrl, gemm_grid(tw->R_cap, N, 128, dev.sms), stream));
+  TW_CUDA(launch_overflow_product(bn1, tm_xo, tm_wu, g1, p1, tw->ctrl, gemm_grid(tw->R_cap, N, bn1, dev.sms), stream));
   TW_CUDA(trace_end(stream, "overflow_up_gemm"));
 
   EpiAccumulateRows::Params p2;
   p2.y = y; p2.slot_row = tw->slot_row; p2.ldy = K; p2.ncols = K;
-  const int ks2 = choose_k_splits(tw->R_cap, K, 256, 2 * N, dev.sms);
-  GemmGeom g2{tw->R_cap, K, 2 * N, tw->ctrl + kCtrlNOver, kGateGroupM, N / kBK, ks2};
+  // The live rows (n_over) are known only on the device: the kernel picks the
+  // number of reduction slices (each at least 8 k-blocks) from them.
+  const int ks2_max = (2 * N / kBK) / 8 > 1 ? (2 * N / kBK) / 8 : 1;
+  GemmGeom g2{tw->R_cap, K, 2 * N, tw->ctrl + kCtrlNOver, kGateGroupM, N / kBK, -ks2_max};
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_overflow_down(tm_ho, tm_wd, g2, p2, tw->ctrl, gemm_grid(tw->R_cap, K, 256, dev.sms, ks2), stream));
+  TW_CUDA(launch_overflow_down(tm_ho, tm_wd, g2, p2, tw->ctrl, gemm_grid(tw->R_cap, K, 256, dev.sms, ks2_max),
+                               stream));
   TW_CUDA(trace_end(stream, "overflow_down_gemm"));
   return TWELL_OK;
 }

@@ -262,23 +262,31 @@ def run_native(args, rank, world, local_rank):
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    traces = []
     launches = 0
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
-            tr = tw.KernelTrace(capacity=8)
-            with tr:
-                starts[i].record()
-                launches += step()
-                ends[i].record()
-            traces.append(tr)
+            starts[i].record()
+            launches += step()
+            ends[i].record()
         torch.cuda.synchronize()
         barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
+
+    # Per-kernel durations: the same K steps again with an event pair around
+    # every kernel (events between kernels stop a launch from overlapping the
+    # previous kernel's tail, so these steps are not the ones timed above).
+    traces = []
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        tr = tw.KernelTrace(capacity=8)
+        with tr:
+            step()
+        traces.append(tr)
+    torch.cuda.synchronize()
     per_kernel = {}
     for tr in traces:
         for name, t in tr.times_ms():
