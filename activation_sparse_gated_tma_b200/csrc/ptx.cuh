@@ -28,7 +28,6 @@ enum : int {
   kCtrlUnitHead = 4,   //   next split-off unit to take
   kCtrlUnitTail = 5,   //   split-off units published
   kCtrlScanned = 6,    //   rows whose units are all published
-  kCtrlEpoch = 7,      //   launch epoch (>= 1): tags row flags and unit records
   kCtrlWords = 64,
 };
 

@@ -11,10 +11,10 @@
 //     active count (the pages report a row maximum above 10x the mean), so a
 //     heavy row is shared by several warps instead of stalling one.
 //   * When the row queue is empty, warps take published units.
-//   * The warp that owns a row (its first unit) stores its partial y_m and
-//     raises the row's flag; warps with later units wait (bounded) for the
-//     flag and add their partial with vector atomics.  The owner was
-//     dequeued before any unit of its row existed, so every wait ends.
+//   * A row that is not split is stored by its warp.  A split row is cleared
+//     by the warp that splits it before its units are published; every unit
+//     (the first one too) then adds its partial y_m with vector atomics, so no
+//     warp ever waits for another.
 // Inside a unit:
 //   * x_m (bf16) and the fp32 partial of y_m stay in registers, spread over the
 //     lanes in 16-byte pieces: lane l holds elements [(j*32 + l)*8, +8).
@@ -46,7 +46,6 @@ struct UpdownParams {
   float* y;
   int* ctrl;
   int4* units;     // [M * N/T] published units {row, tile begin, tile end, unused}
-  int* row_flag;   // [M] epoch at which the row's owner stored its partial
   int stages;
 };
 
@@ -74,24 +73,35 @@ __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   return pol;
 }
 
-// 1-D bulk copy global -> shared (no multicast), completion on an mbarrier.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,
-                                          uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-          smem_u32(smem_dst)),
-      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
+// 16-byte asynchronous copy global -> shared (bypassing L1), with an L2
+// cache-policy hint.  Completion is tracked per thread with commit/wait groups.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Wait until at most n of this thread's committed groups are still pending.
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 5: cp_async_wait<5>(); break;
+    default: cp_async_wait<6>(); break;
+  }
 }
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
-}
-
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
@@ -104,21 +114,20 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
 }
 
 // Shared memory of one warp: [ring: stages x (2K bf16 W_u row | 2K bf16 W_d row)]
-// [list n: int x cap][list g: float x cap][mbarriers: stages].
+// [list n: int x cap][list g: float x cap].
 __host__ __device__ constexpr size_t updown_warp_bytes(int K, int stages) {
-  return ((static_cast<size_t>(stages) * 4 * K + kUpdownListCap * 8 + stages * 8) + 127) / 128 * 128;
+  return ((static_cast<size_t>(stages) * 4 * K + kUpdownListCap * 8) + 127) / 128 * 128;
 }
 
-// Per-warp streaming state.
+// Per-warp streaming state.  The ring is lane-private in effect: lane l
+// copies, and later reads, only the 16-byte pieces l, l + 32, l + 64, ... of
+// every row it holds, so no lane ever waits for another lane's copies.
 struct WarpRing {
   uint8_t* ring;
   int* list_n;
   float* list_g;
-  uint64_t* bars;
   uint32_t slot_bytes;
-  int stages;
-  int head;             // ring slot of the next entry
-  uint32_t head_phase;  // parity that slot's mbarrier completes next
+  int stages;  // >= 2
   uint64_t policy;
 };
 
@@ -154,12 +163,21 @@ __device__ __forceinline__ int list_entries(const UpdownParams& p, const WarpRin
   return E;
 }
 
-__device__ __forceinline__ void issue_entry(const UpdownParams& p, WarpRing& w, int slot, int e) {
-  const int n = w.list_n[e];
-  uint8_t* dst = w.ring + static_cast<size_t>(slot) * w.slot_bytes;
-  mbar_arrive_expect_tx(&w.bars[slot], w.slot_bytes);
-  bulk_load(dst, p.wu_t + static_cast<int64_t>(n) * p.K, w.slot_bytes / 2, &w.bars[slot], w.policy);
-  bulk_load(dst + w.slot_bytes / 2, p.wd + static_cast<int64_t>(n) * p.K, w.slot_bytes / 2, &w.bars[slot], w.policy);
+// This lane's pieces of W_u^T[n] and W_d[n] into ring slot `slot`.
+template <int KV>
+__device__ __forceinline__ void issue_entry(const UpdownParams& p, const WarpRing& w, int slot, int n, int lane) {
+  uint4* dst = reinterpret_cast<uint4*>(w.ring + static_cast<size_t>(slot) * w.slot_bytes);
+  const uint4* su = reinterpret_cast<const uint4*>(p.wu_t + static_cast<int64_t>(n) * p.K);
+  const uint4* sd = reinterpret_cast<const uint4*>(p.wd + static_cast<int64_t>(n) * p.K);
+  const int kv = p.K / 8;
+#pragma unroll
+  for (int j = 0; j < KV; ++j) {
+    const int v = j * 32 + lane;
+    if (v < kv) {
+      cp_async16(dst + v, su + v, w.policy);
+      cp_async16(dst + kv + v, sd + v, w.policy);
+    }
+  }
 }
 
 // s[e] += the products of the e-th bf16 pair of a and b: four independent
@@ -181,40 +199,27 @@ __device__ __forceinline__ void dot8_acc4(const uint4& a, const uint4& b, float 
   }
 }
 
-// Streams the E listed entries through the ring and accumulates them.  Entries
+// Streams the E listed entries through the ring and accumulates them.  Every
+// ring slot is one copy group per lane: the first `stages` entries are put in
+// flight, and each consumed slot is refilled with the entry `stages` places
+// ahead (an empty group past the end keeps the group count uniform).  Entries
 // are taken two at a time: the two dot products (four partial sums each), their
 // shuffle reductions and the two accumulations are independent, so each warp
 // keeps several short dependency chains in flight instead of one long one.
 template <int KV>
-__device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& w, int E, const uint4 (&xv)[KV],
+__device__ __forceinline__ void stream_entries(const UpdownParams& p, const WarpRing& w, int E, const uint4 (&xv)[KV],
                                                float (&acc)[KV][8], int lane) {
-  const int pre = min(w.stages, E);
-  if (lane == 0) {
-    int s = w.head;
-    for (int e = 0; e < pre; ++e) {
-      issue_entry(p, w, s, e);
-      if (++s == w.stages) s = 0;
-    }
+  const int S = w.stages;
+  for (int e = 0; e < S; ++e) {
+    if (e < E) issue_entry<KV>(p, w, e, w.list_n[e], lane);
+    cp_async_commit();
   }
   auto slot = [&](int s) { return reinterpret_cast<const uint4*>(w.ring + static_cast<size_t>(s) * w.slot_bytes); };
+  int sa = 0;
   for (int e = 0; e < E; e += 2) {
     const bool two = e + 1 < E;
-    const int sa = w.head;
-    const uint32_t pa = w.head_phase;
-    const int sb = sa + 1 == w.stages ? 0 : sa + 1;
-    const uint32_t pb = sa + 1 == w.stages ? (pa ^ 1u) : pa;
-    bool ok = mbar_wait(&w.bars[sa], pa, p.ctrl);
-    if (ok && two) ok = mbar_wait(&w.bars[sb], pb, p.ctrl);
-    if (!ok) {
-      // Let the copies still in flight land before the CTA may exit (bounded).
-      int s2 = sa;
-      uint32_t ph = pa;
-      for (int e2 = e; e2 < min(E, e + w.stages); ++e2) {
-        mbar_wait(&w.bars[s2], ph, p.ctrl);
-        if (++s2 == w.stages) { s2 = 0; ph ^= 1u; }
-      }
-      return false;
-    }
+    const int sb = sa + 1 == S ? 0 : sa + 1;
+    cp_async_wait_pending(S - 2);  // this lane's pieces of entries e and e + 1 have landed
     const uint4* ua = slot(sa);
     const uint4* ub = slot(sb);
     float qa[4] = {0.f, 0.f, 0.f, 0.f}, qb[4] = {0.f, 0.f, 0.f, 0.f};
@@ -243,15 +248,13 @@ __device__ __forceinline__ bool stream_entries(const UpdownParams& p, WarpRing& 
         if (two) axpy8_bf16(acc[j], hb, db[j * 32 + lane]);
       }
     }
-    __syncwarp();  // every lane's reads of the two slots are done before they are refilled
-    // Lanes 0 and 1 refill the two slots in one instruction.
-    const int refill = e + (lane & 1) + w.stages;
-    if (lane < (two ? 2 : 1) && refill < E) issue_entry(p, w, lane == 0 ? sa : sb, refill);
-    const int used = two ? 2 : 1;
-    w.head += used;
-    if (w.head >= w.stages) { w.head -= w.stages; w.head_phase ^= 1u; }
+    // The two slots were read (by this lane) above; refill them.
+    if (e + S < E) issue_entry<KV>(p, w, sa, w.list_n[e + S], lane);
+    cp_async_commit();
+    if (e + 1 + S < E) issue_entry<KV>(p, w, sb, w.list_n[e + 1 + S], lane);
+    cp_async_commit();
+    sa = sb + 1 == S ? 0 : sb + 1;
   }
-  return true;
 }
 
 template <int KV>
@@ -264,6 +267,20 @@ __device__ __forceinline__ void load_x(const UpdownParams& p, int row, uint4 (&x
     xv[j] = k0 < p.K ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+  }
+}
+
+template <int KV>
+__device__ __forceinline__ void zero_y(const UpdownParams& p, int row, int lane) {
+  float* yr = p.y + static_cast<int64_t>(row) * p.K;
+#pragma unroll
+  for (int j = 0; j < KV; ++j) {
+    const int k0 = (j * 32 + lane) * 8;
+    if (k0 < p.K) {
+      float4* dst = reinterpret_cast<float4*>(yr + k0);
+      dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      dst[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 }
 
@@ -320,19 +337,10 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
   w.ring = smem + static_cast<size_t>(warp) * updown_warp_bytes(p.K, p.stages);
   w.list_n = reinterpret_cast<int*>(w.ring + static_cast<size_t>(p.stages) * w.slot_bytes);
   w.list_g = reinterpret_cast<float*>(w.list_n + kUpdownListCap);
-  w.bars = reinterpret_cast<uint64_t*>(w.list_g + kUpdownListCap);
-  w.head = 0;
-  w.head_phase = 0;
-  if (lane == 0) {
-    for (int s = 0; s < p.stages; ++s) mbar_init(&w.bars[s], 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
   w.policy = l2_evict_last_policy();
   // Set-up above overlaps the previous kernel (programmatic dependent launch).
   griddep_launch_dependents();
   griddep_wait();
-  const int epoch = ld_acquire(ctrl + kCtrlEpoch);
 
   uint4 xv[KV];
   float acc[KV][8];
@@ -369,25 +377,20 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
       for (int k = 1 + lane; k < nunits; k += 32)
         p.units[base + k - 1] = make_int4(row, unit_cut(w.list_n, NT, total, nunits, k),
                                           unit_cut(w.list_n, NT, total, nunits, k + 1), 0);
+      // Every unit of a split row adds into y_m: clear it before any unit is taken.
+      zero_y<KV>(p, row, lane);
+      __threadfence();
     }
     __syncwarp();
-    if (lane == 0) {
-      __threadfence();
-      atomicAdd(ctrl + kCtrlScanned, 1);
-    }
+    if (lane == 0) atomicAdd(ctrl + kCtrlScanned, 1);
 
     int cursor = 0;
     while (ok && cursor < own_end) {
       const int E = list_entries(p, w, row, cursor, own_end, lane);
-      if (E > 0) ok = stream_entries<KV>(p, w, E, xv, acc, lane);
+      if (E > 0) stream_entries<KV>(p, w, E, xv, acc, lane);
     }
     if (!ok) break;
-    write_y<KV>(p, row, acc, false, lane);
-    if (nunits > 1) {
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release(p.row_flag + row, epoch);
-    }
+    write_y<KV>(p, row, acc, nunits > 1, lane);
   }
 
   // ---------------------------------------------------------------- split-off units
@@ -433,28 +436,13 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
     while (ok && cursor < te) {
       const int E = list_entries(p, w, row, cursor, te, lane);
       listed += E;
-      if (E > 0) ok = stream_entries<KV>(p, w, E, xv, acc, lane);
+      if (E > 0) stream_entries<KV>(p, w, E, xv, acc, lane);
     }
     if (!ok) break;
-    if (listed == 0) continue;
-    // Add after the row's owner has stored its partial (bounded wait).
-    int flag_ok = 1;
-    if (lane == 0) {
-      const unsigned long long t0 = global_ns();
-      while (ld_acquire(p.row_flag + row) != epoch) {
-        if (global_ns() - t0 > kWaitLimitNs) {
-          set_flag(ctrl, kFlagWaitTimeout);
-          flag_ok = 0;
-          break;
-        }
-      }
-    }
-    flag_ok = __shfl_sync(0xffffffffu, flag_ok, 0);
-    if (!flag_ok) break;
-    write_y<KV>(p, row, acc, true, lane);
+    if (listed > 0) write_y<KV>(p, row, acc, true, lane);
   }
 
-  // The last warp out rewinds the queues and opens the next epoch.
+  // The last warp out rewinds the queues for the next launch.
   if (lane == 0) {
     __threadfence();
     const int total = gridDim.x * (blockDim.x >> 5);
@@ -463,7 +451,6 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
       ctrl[kCtrlUnitHead] = 0;
       ctrl[kCtrlUnitTail] = 0;
       ctrl[kCtrlScanned] = 0;
-      ctrl[kCtrlEpoch] = epoch + 1;
       __threadfence();
       ctrl[kCtrlDone] = 0;
     }

@@ -135,7 +135,7 @@ twell_status tmap_bf16(const void* ptr, uint64_t inner, uint64_t outer, uint32_t
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, units, row_flag, total;
+  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, units, total;
 };
 
 bool shape_ok(int M, int K, int N, int T, int C, int R_cap) {
@@ -158,7 +158,6 @@ Layout layout(int M, int K, int N, int T, int C, int R_cap) {
   L.x_over = o; o = align256(o + size_t(R_cap) * K * 2);
   L.h_over = o; o = align256(o + size_t(R_cap) * N * 4);
   L.units = o; o = align256(o + size_t(M) * NT * 16);
-  L.row_flag = o; o = align256(o + size_t(M) * 4);
   L.total = o;
   return L;
 }
@@ -167,24 +166,19 @@ twell_status check_buf(const twell_buf* tw) {
   if (!tw) return fail(TWELL_ERR_INVALID, "twell_buf is NULL");
   if (!shape_ok(tw->M, tw->K, tw->N, tw->T, tw->C, tw->R_cap)) return fail(TWELL_ERR_INVALID, "twell_buf has invalid sizes");
   if (!tw->counts || !tw->idx || !tw->vals || !tw->dense_rows || !tw->row_slot || !tw->slot_row || !tw->ctrl ||
-      !tw->x_over || !tw->h_over || !tw->units || !tw->row_flag)
+      !tw->x_over || !tw->h_over || !tw->units)
     return fail(TWELL_ERR_INVALID, "twell_buf is not initialised");
   return TWELL_OK;
 }
 
 // ---------------------------------------------------------------- small kernels
 // Start of a gate pass: no row holds a dense-row slot, control words at zero.
-// The fused kernel's epoch starts at 1 so that zeroed row flags mean "not stored".
-__global__ void twell_reset_kernel(int* __restrict__ row_slot, int* __restrict__ row_flag, int M,
-                                   int* __restrict__ ctrl) {
+__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl) {
   griddep_launch_dependents();
   griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < kCtrlWords) ctrl[i] = (i == kCtrlEpoch) ? 1 : 0;
-  for (int r = i; r < M; r += gridDim.x * blockDim.x) {
-    row_slot[r] = kSlotFree;
-    row_flag[r] = 0;
-  }
+  if (i < kCtrlWords) ctrl[i] = 0;
+  for (int r = i; r < M; r += gridDim.x * blockDim.x) row_slot[r] = kSlotFree;
 }
 
 // Warps per CTA and ring depth of the fused kernel for a given K: eight warps
@@ -215,7 +209,7 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
   p.x = x; p.wu_t = wu_t; p.wd = wd;
   p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals;
   p.M = tw->M; p.K = tw->K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
-  p.y = y; p.ctrl = tw->ctrl; p.units = reinterpret_cast<int4*>(tw->units); p.row_flag = tw->row_flag;
+  p.y = y; p.ctrl = tw->ctrl; p.units = reinterpret_cast<int4*>(tw->units);
   p.stages = stages;
   return launch_pdl(twell_updown_kernel<KV>, sms, 32 * warps, smem, s, p);
 }
@@ -313,7 +307,6 @@ twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int 
   tw->x_over = reinterpret_cast<uint16_t*>(b + L.x_over);
   tw->h_over = reinterpret_cast<uint16_t*>(b + L.h_over);
   tw->units = b + L.units;
-  tw->row_flag = reinterpret_cast<int32_t*>(b + L.row_flag);
   tw->M = M; tw->K = K; tw->N = N; tw->T = T; tw->C = C; tw->R_cap = R_cap;
   return TWELL_OK;
 }
@@ -338,8 +331,7 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
 
   const int rgrid = static_cast<int>((static_cast<int64_t>(M) + 255) / 256 < 1024 ? (M + 255) / 256 : 1024);
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, stream, tw->row_slot, tw->row_flag, M,
-                     tw->ctrl));
+  TW_CUDA(launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, stream, tw->row_slot, M, tw->ctrl));
   TW_CUDA(trace_end(stream, "twell_reset"));
 
   GateTwellParams p;

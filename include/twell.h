@@ -69,13 +69,12 @@ typedef enum {
  *                                 -2 = needed but R_cap was exhausted
  *   slot_row   int32  [R_cap]     row that owns each slot (valid for slots < n_over)
  *   ctrl       int32  [64]        device control words: [0] n_over (rows that
- *                                 asked for a slot), [1] status flags, [2..3]
- *                                 work-queue counters
+ *                                 asked for a slot), [1] status flags, [2..6]
+ *                                 work-queue counters of the fused kernel
  *   x_over     bf16   [R_cap][K]  scratch: gathered x rows of slotted rows
  *   h_over     bf16   [R_cap][2N] scratch: overflow-tile hidden activations as
  *                                 bf16 hi (columns < N) + lo (columns >= N) parts
  *   units      int32  [M*NT][4]   scratch: work units of rows split across warps
- *   row_flag   int32  [M]         scratch: per-row publication flags of the fused kernel
  */
 typedef struct twell_buf {
   uint16_t* counts;
@@ -88,7 +87,6 @@ typedef struct twell_buf {
   uint16_t* x_over;
   uint16_t* h_over;
   void* units;
-  int32_t* row_flag;
   int M, K, N, T, C, R_cap;
 } twell_buf;
 

@@ -49,7 +49,7 @@ def test_buf_init_layout_is_aligned_and_disjoint():
     NT = N // T
     spans = [("ctrl", 64 * 4), ("counts", M * NT * 2), ("idx", M * NT * C), ("vals", M * NT * C * 4),
              ("row_slot", M * 4), ("slot_row", R * 4), ("dense_rows", R * N * 4), ("x_over", R * K * 2),
-             ("h_over", R * N * 4), ("units", M * NT * 16), ("row_flag", M * 4)]
+             ("h_over", R * N * 4), ("units", M * NT * 16)]
     ranges = []
     for name, size in spans:
         p = getattr(b, name)
