@@ -149,9 +149,30 @@ __device__ __forceinline__ int list_entries(const UpdownParams& p, const WarpRin
     if (lane < k && ce > 0) {
       const int64_t rec = (static_cast<int64_t>(row) * NT + t) * p.C;
       const int off = E + incl - ce;
-      for (int s = 0; s < ce; ++s) {
-        w.list_n[off + s] = t * p.T + p.idx[rec + s];
-        w.list_g[off + s] = p.vals[rec + s];
+      const int nbase = t * p.T;
+      if ((p.C & 7) == 0) {
+        // Eight slots per step: one 8-byte and two 16-byte loads, all issued
+        // before the first store (records are 8-slot aligned when C % 8 == 0).
+#pragma unroll 1
+        for (int s0 = 0; s0 < ce; s0 += 8) {
+          const uint2 iv = *reinterpret_cast<const uint2*>(p.idx + rec + s0);
+          const float4 v0 = *reinterpret_cast<const float4*>(p.vals + rec + s0);
+          const float4 v1 = *reinterpret_cast<const float4*>(p.vals + rec + s0 + 4);
+          const float g[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            if (s0 + s < ce) {
+              const uint32_t word = s < 4 ? iv.x : iv.y;
+              w.list_n[off + s0 + s] = nbase + static_cast<int>((word >> (8 * (s & 3))) & 0xFFu);
+              w.list_g[off + s0 + s] = g[s];
+            }
+          }
+        }
+      } else {
+        for (int s = 0; s < ce; ++s) {
+          w.list_n[off + s] = nbase + p.idx[rec + s];
+          w.list_g[off + s] = p.vals[rec + s];
+        }
       }
     }
     if (k > 0) E += __shfl_sync(0xffffffffu, incl, k - 1);
