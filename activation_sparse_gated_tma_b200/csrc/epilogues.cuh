@@ -52,6 +52,8 @@ __device__ __forceinline__ float relu_f(float z) { return z > 0.f ? z : 0.f; }
 // before the accumulator is ready; run() consumes it.  Most epilogues need none.
 struct EpiNoPrepare {
   template <int BN>
+  static constexpr int kWarps = 4;  // epilogue warps (4, or 8 to split the columns)
+  template <int BN>
   struct Pre {};
   template <int BN, class Params>
   static __device__ __forceinline__ void prepare(const Params&, Pre<BN>&, int, int, int) {}
@@ -82,16 +84,20 @@ struct EpiGateTwell : EpiNoPrepare {
   // [column][lane] so that every thread's dynamically indexed reads of its own
   // row hit distinct banks.
   static constexpr int kScratchBytes = 32 * 32 * 4;
+  // Two TwELL tiles per CTA tile: eight warps, one TwELL tile each per row.
+  template <int BN>
+  static constexpr int kWarps = BN / T >= 2 ? 8 : 4;
 
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
-                                             int nb, int lane, int* ctrl, void* scratch) {
+                                             int nb, int lane, int* ctrl, void* scratch, int part, int nparts) {
     static_assert(BN % T == 0, "a CTA tile must hold whole TwELL tiles");
     float* stage = static_cast<float*>(scratch) + lane;
     const bool valid = row < m_rows;
     const int NT = p.N / T;
+    constexpr int kSub = BN / T;  // TwELL tiles in the CTA tile
 #pragma unroll 1
-    for (int st = 0; st < BN / T; ++st) {
+    for (int st = part * kSub / nparts; st < (part + 1) * kSub / nparts; ++st) {
       const int t = nb * (BN / T) + st;
       const uint32_t tcol = taddr + st * T;
       const int64_t rec = static_cast<int64_t>(row) * NT + t;
@@ -170,7 +176,7 @@ struct EpiGatedProduct : EpiNoPrepare {
   };
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
-                                             int nb, int, int*, void*) {
+                                             int nb, int, int*, void*, int, int) {
     const bool valid = row < m_rows;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
@@ -209,7 +215,7 @@ struct EpiStoreF32 : EpiNoPrepare {
   };
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
-                                             int nb, int, int*, void*) {
+                                             int nb, int, int*, void*, int, int) {
     const bool valid = row < m_rows;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
@@ -253,6 +259,8 @@ struct EpiStoreF32 : EpiNoPrepare {
 // second stage keeps ~16 bits of h while feeding bf16 tensor cores.
 struct EpiOverflowProduct {
   static constexpr int kScratchBytes = 0;
+  template <int BN>
+  static constexpr int kWarps = 4;
   struct Params {
     const uint16_t* counts;   // [M][N/T]
     const float* dense_rows;  // [R_cap][N]
@@ -285,7 +293,7 @@ struct EpiOverflowProduct {
   }
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, const Pre<BN>& pre, uint32_t taddr, int row, int m_rows,
-                                             int nb, int, int*, void*) {
+                                             int nb, int, int*, void*, int, int) {
     const bool valid = row < m_rows;
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) {
@@ -328,7 +336,7 @@ struct EpiAccumulateRows : EpiNoPrepare {
   };
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
-                                             int nb, int, int*, void*) {
+                                             int nb, int, int*, void*, int, int) {
     const int m = row < m_rows ? p.slot_row[row] : -1;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {

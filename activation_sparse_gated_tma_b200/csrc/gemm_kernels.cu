@@ -9,14 +9,15 @@ namespace {
 template <int BN, bool B_MN, bool DUAL, int STAGES, class Epi>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmGeom& g,
                    const typename Epi::Params& ep, int* ctrl, int grid, cudaStream_t s) {
-  constexpr size_t smem = gemm_smem_bytes<BN, DUAL, STAGES, Epi::kScratchBytes>();
+  constexpr int warps = Epi::template kWarps<BN>;
+  constexpr size_t smem = gemm_smem_bytes<BN, DUAL, STAGES, Epi::kScratchBytes, warps>();
   static_assert(smem <= 232448, "exceeds the 227 KB per-CTA shared memory limit");
   auto kern = tc_gemm_kernel<BN, B_MN, DUAL, STAGES, Epi>;
   // The attribute is per device; setting it is cheap and idempotent.
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaSuccess;
-  return launch_pdl(kern, grid, kGemmThreads, smem, s, a, b, b2, g, ep, ctrl);
+  return launch_pdl(kern, grid, gemm_threads<Epi, BN>(), smem, s, a, b, b2, g, ep, ctrl);
 }
 
 }  // namespace

@@ -9,9 +9,11 @@
 // One CTA per SM, 192 threads:
 //   warp 0      TMA producer (one elected lane) filling a STAGES-deep smem ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..5  epilogue: thread i of warp w owns TMEM lane 32*(w%4)+i, i.e.
-//               one output row of the 128-row tile; per tile it runs
-//               Epi::prepare (before the accumulator is ready) and Epi::run.
+//   warps 2..   epilogue (4 or 8 warps, Epi::kWarps): thread i of warp w owns
+//               TMEM lane 32*(w%4)+i, i.e. one output row of the 128-row tile
+//               (with 8 warps, two warps share a row and split its columns);
+//               per tile it runs Epi::prepare (before the accumulator is
+//               ready) and Epi::run.
 // Accumulators are double-buffered in TMEM so the epilogue of tile i overlaps
 // the MMAs of tile i+1.  Every wait is bounded (see mbar_wait).
 #pragma once
@@ -25,7 +27,11 @@ namespace twell {
 constexpr int kBM = 128;      // UMMA M (rows per tile, = TMEM lanes)
 constexpr int kBK = 64;       // bf16 elements per 128-byte swizzle row
 constexpr int kUmmaK = 16;    // K per tcgen05.mma kind::f16
-constexpr int kGemmThreads = 192;
+// Threads of a CTA: warp 0 (TMA), warp 1 (TMEM + MMA) and the epilogue warps.
+template <class Epi, int BN>
+constexpr int gemm_threads() {
+  return 64 + 32 * Epi::template kWarps<BN>;
+}
 
 struct GemmGeom {
   int M;                    // rows of A and D
@@ -51,11 +57,11 @@ struct GemmSmem {
 };
 
 // Shared memory of one CTA: the operand ring, the barriers, and EPI_SCRATCH
-// bytes of private scratch for each of the four epilogue warps.
-template <int BN, bool DUAL, int STAGES, int EPI_SCRATCH>
+// bytes of private scratch for each of the EPI_WARPS epilogue warps.
+template <int BN, bool DUAL, int STAGES, int EPI_SCRATCH, int EPI_WARPS>
 constexpr size_t gemm_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * GemmSmem<BN, DUAL>::kStageBytes +
-         (2 * STAGES + 4) * sizeof(uint64_t) + 16 + 128 + 4 * static_cast<size_t>(EPI_SCRATCH);
+         (2 * STAGES + 4) * sizeof(uint64_t) + 16 + 128 + EPI_WARPS * static_cast<size_t>(EPI_SCRATCH);
 }
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int& mb, int& nb) {
@@ -69,7 +75,7 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int 
 }
 
 template <int BN, bool B_MN, bool DUAL, int STAGES, class Epi>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<Epi, BN>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const GemmGeom g, const typename Epi::Params ep,
                    int* ctrl) {
@@ -94,7 +100,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * Epi::template kWarps<BN>);
     }
     fence_barrier_init();
   }
@@ -206,6 +212,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const int row_in_tile = q * 32 + lane;
+    // With eight epilogue warps every quadrant has two; `part` says which half
+    // of the tile's columns (as the epilogue divides them) this warp takes.
+    constexpr int kParts = Epi::template kWarps<BN> / 4;
+    const int part = (warp - 2) >> 2;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       int mb, nb;
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
       Epi::template run<BN>(ep, pre, taddr, mb * kBM + row_in_tile, m_rows, nb, lane, ctrl,
-                            epi_scratch + (warp - 2) * Epi::kScratchBytes);
+                            epi_scratch + (warp - 2) * Epi::kScratchBytes, part, kParts);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

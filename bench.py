@@ -55,11 +55,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; a profile taken on other sources is stale."""
+# The sources each profiled kernel is built from (its launch configuration
+# lives in twell_api.cu, so that file counts for every kernel).
+KERNEL_SOURCES = {
+    "twell_updown": ("sparse_updown.cuh", "ptx.cuh", "twell_api.cu"),
+    "gate_twell_gemm": ("tc_gemm.cuh", "epilogues.cuh", "gemm_kernels.cu", "internal.h", "ptx.cuh", "twell_api.cu"),
+    "overflow_up_gemm": ("tc_gemm.cuh", "epilogues.cuh", "gemm_kernels.cu", "internal.h", "ptx.cuh", "twell_api.cu"),
+    "overflow_down_gemm": ("tc_gemm.cuh", "epilogues.cuh", "gemm_kernels.cu", "internal.h", "ptx.cuh", "twell_api.cu"),
+}
+
+
+def kernel_source_hash(kernel: str = "") -> str:
+    """Hash of the CUDA sources of `kernel` (all sources if unknown); a profile
+    taken on other sources is stale."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "activation_sparse_gated_tma_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc))
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -74,7 +86,7 @@ def profiled_traffic(kernel: str, workload: str):
     text = open(path).read()
     m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(kernel):
         return None
     return float(m_bytes.group(1))
 
