@@ -193,6 +193,25 @@ def cpu_oracle_rate(d, w, rows_target_s: float, min_rows: int = 8):
     return rows.size / dt, int(rows.size), dt, nthreads
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise maximum of per-rank timings over all ranks (one all-reduce;
+    every rank must call it).  With one rank the values come back unchanged."""
+    values = [float(v) for v in values]
+    if world <= 1:
+        return values
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world: int, rows_per_rank: int, ms: float) -> float:
+    """Tokens/s of the whole job: every rank's rows over the slowest rank's time."""
+    return world * rows_per_rank / (ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     if rank != 0:
@@ -305,10 +324,6 @@ def run_native(args, rank, world, local_rank):
             per_kernel.setdefault(name, []).append(t)
     kern_ms = {k: sum(v) / len(v) for k, v in per_kernel.items()}
 
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
 
     # In-build dense tcgen05 FFN on the same inputs (same flush discipline).
     h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
@@ -324,10 +339,6 @@ def run_native(args, rank, world, local_rank):
         b.synchronize()
         dense_ms.append(a.elapsed_time(b))
     dense_ms = sum(dense_ms) / len(dense_ms)
-    if world > 1:
-        t = torch.tensor([dense_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        dense_ms = float(t.item())
 
     # End to end through the public API with host buffers: pinned x in, y out.
     x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -352,11 +363,9 @@ def run_native(args, rank, world, local_rank):
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
     e2e_ms = sum(e2e_ms) / len(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
 
+    # One collective on every rank: the job's time is the slowest rank's.
+    ms, dense_ms, e2e_ms = max_over_ranks([ms, dense_ms, e2e_ms], world, dev)
     if rank != 0:
         return
 
@@ -399,7 +408,7 @@ def run_native(args, rank, world, local_rank):
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{rows} seeded rows of {w.M} ({sec:.1f} s): fp64 gate, TwELL pack, sparse y"}
 
-    value = world * M / (ms * 1e-3)
+    value = job_throughput(world, M, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -415,10 +424,10 @@ def run_native(args, rank, world, local_rank):
                           >= bytes_path / (peaks["hbm_gbs"] * 1e9) else "hbm",
                           "flops": flops_gate + flops_over, "bytes": bytes_path},
         "kernels": kernels,
-        "dense": {"ms_per_step": dense_ms, "value": world * M / (dense_ms * 1e-3), "unit": UNIT},
+        "dense": {"ms_per_step": dense_ms, "value": job_throughput(world, M, dense_ms), "unit": UNIT},
         "speedup_vs_dense": dense_ms / ms,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * M / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": 2 * M * K,
+        "e2e": {"value": job_throughput(world, M, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * M * K,
                 "d2h_bytes_per_step": 4 * M * K, "ms_per_step": e2e_ms},
         "gpu_launches": launches,
         "clocks": clk.summary(),
