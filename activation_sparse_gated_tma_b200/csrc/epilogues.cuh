@@ -130,6 +130,9 @@ struct EpiGateTwell : EpiNoPrepare {
       }
       if (valid) p.counts[rec] = static_cast<uint16_t>(cnt);
       const bool ov = valid && cnt > p.C;
+      // Entries the fused kernel will stream (it sizes its work units from the total).
+      const int listed = warp_sum_int(ov ? 0 : cnt);
+      if (lane == 0 && listed > 0) atomicAdd(ctrl + kCtrlEntries, listed);
       if (__any_sync(0xffffffffu, ov)) {
         int slot = -1;
         bool fresh = false;

@@ -28,6 +28,7 @@ enum : int {
   kCtrlUnitHead = 4,   //   next split-off unit to take
   kCtrlUnitTail = 5,   //   split-off units published
   kCtrlScanned = 6,    //   rows whose units are all published
+  kCtrlEntries = 7,    // TwELL entries listed by the gate pass (non-overflow tiles)
   kCtrlWords = 64,
 };
 
@@ -202,6 +203,12 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(float_to_bf16_bits(lo)) | (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -5,8 +5,8 @@
 //
 // Work distribution (persistent grid, one CTA per SM, warps independent):
 //   * A warp takes the next token row from a queue.  It scans the row's TwELL
-//     counts; if the row holds more than kUnitCap entries it cuts the row's
-//     tile range into units of about kUnitCap entries, keeps the first unit
+//     counts; if the row holds more than unit_cap entries it cuts the row's
+//     tile range into units of about unit_cap entries, keeps the first unit
 //     and publishes the others on a second queue.  Rows are 100x apart in
 //     active count (the pages report a row maximum above 10x the mean), so a
 //     heavy row is shared by several warps instead of stalling one.
@@ -32,8 +32,8 @@
 
 namespace twell {
 
-constexpr int kUpdownListCap = 256;  // list entries per warp and segment (also the N/T limit)
-constexpr int kUnitCap = 16;         // target entries per unit of a split row
+constexpr int kUpdownListCap = 256;  // largest list of a warp (entries per segment; also the N/T limit)
+constexpr int kUnitCap = 16;         // largest target entries per unit of a split row
 
 struct UpdownParams {
   const uint16_t* x;
@@ -47,7 +47,15 @@ struct UpdownParams {
   int* ctrl;
   int4* units;     // [M * N/T] published units {row, tile begin, tile end, unused}
   int stages;
+  int list_cap;    // list entries per warp: >= N/T and >= C
 };
+
+// Warps per CTA: twelve for K <= 1536 (the state of a warp fits 170
+// registers), else eight.
+template <int KV>
+constexpr int updown_max_warps() {
+  return KV <= 6 ? 12 : 8;
+}
 
 // acc += h * d for 8 bf16 elements of d, as four packed fp32x2 FMAs (each lane
 // of a pair rounds exactly as a scalar fp32 FMA would).
@@ -115,8 +123,8 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
 
 // Shared memory of one warp: [ring: stages x (2K bf16 W_u row | 2K bf16 W_d row)]
 // [list n: int x cap][list g: float x cap].
-__host__ __device__ constexpr size_t updown_warp_bytes(int K, int stages) {
-  return ((static_cast<size_t>(stages) * 4 * K + kUpdownListCap * 8) + 127) / 128 * 128;
+__host__ __device__ constexpr size_t updown_warp_bytes(int K, int stages, int list_cap) {
+  return ((static_cast<size_t>(stages) * 4 * K + static_cast<size_t>(list_cap) * 8) + 127) / 128 * 128;
 }
 
 // Per-warp streaming state.  The ring is lane-private in effect: lane l
@@ -126,6 +134,7 @@ struct WarpRing {
   uint8_t* ring;
   int* list_n;
   float* list_g;
+  int list_cap;
   uint32_t slot_bytes;
   int stages;  // >= 2
   uint64_t policy;
@@ -144,7 +153,7 @@ __device__ __forceinline__ int list_entries(const UpdownParams& p, const WarpRin
     const int c = t < te ? static_cast<int>(crow[t]) : 0;
     const int ce = (c > 0 && c <= p.C) ? c : 0;
     const int incl = warp_inclusive_scan(ce, lane);
-    const uint32_t fit = __ballot_sync(0xffffffffu, E + incl <= kUpdownListCap);
+    const uint32_t fit = __ballot_sync(0xffffffffu, E + incl <= w.list_cap);
     const int k = __popc(fit);  // fitting lanes form a prefix: incl is non-decreasing
     if (lane < k && ce > 0) {
       const int64_t rec = (static_cast<int64_t>(row) * NT + t) * p.C;
@@ -345,7 +354,7 @@ __device__ __forceinline__ int unit_cut(const int* prefix, int NT, int total, in
 }
 
 template <int KV>
-__global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams p) {
+__global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_kernel(const UpdownParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -355,13 +364,20 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
   WarpRing w;
   w.slot_bytes = 4u * p.K;
   w.stages = p.stages;
-  w.ring = smem + static_cast<size_t>(warp) * updown_warp_bytes(p.K, p.stages);
+  w.ring = smem + static_cast<size_t>(warp) * updown_warp_bytes(p.K, p.stages, p.list_cap);
   w.list_n = reinterpret_cast<int*>(w.ring + static_cast<size_t>(p.stages) * w.slot_bytes);
-  w.list_g = reinterpret_cast<float*>(w.list_n + kUpdownListCap);
+  w.list_g = reinterpret_cast<float*>(w.list_n + p.list_cap);
+  w.list_cap = p.list_cap;
   w.policy = l2_evict_last_policy();
   // Set-up above overlaps the previous kernel (programmatic dependent launch).
   griddep_launch_dependents();
   griddep_wait();
+
+  // Units of about total entries / warps entries when that is below
+  // kUnitCap: with few rows, heavy rows are cut finer so that every warp
+  // streams; never below 2 entries, whose fixed cost would dominate.
+  int unit_cap = ld_acquire(ctrl + kCtrlEntries) / static_cast<int>(gridDim.x * (blockDim.x >> 5));
+  unit_cap = unit_cap < 2 ? 2 : (unit_cap > kUnitCap ? kUnitCap : unit_cap);
 
   uint4 xv[KV];
   float acc[KV][8];
@@ -387,7 +403,7 @@ __global__ void __launch_bounds__(256, 1) twell_updown_kernel(const UpdownParams
       total += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncwarp();
-    int nunits = (total + kUnitCap - 1) / kUnitCap;
+    int nunits = (total + unit_cap - 1) / unit_cap;
     if (nunits > NT) nunits = NT;
     if (nunits < 1) nunits = 1;
     const int own_end = unit_cut(w.list_n, NT, total, nunits, 1);

@@ -181,27 +181,44 @@ __global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __res
   for (int r = i; r < M; r += gridDim.x * blockDim.x) row_slot[r] = kSlotFree;
 }
 
-// Warps per CTA and ring depth of the fused kernel for a given K: eight warps
-// when each can keep at least two entries in flight, else four.
-void updown_config(int K, int& warps, int& stages) {
+// Launch shape of the fused kernel.
+struct UpdownShape {
+  int warps, stages, list_cap;
+};
+
+// Twelve warps (K <= 1536) with a list just large enough (>= N/T, >= C, >= 96
+// entries) when each warp still gets three ring stages; else eight warps with
+// the full list when each gets two; else four.
+UpdownShape updown_shape(int K, int NT, int C, int max_warps) {
   constexpr size_t kBudget = 232448;  // 227 KB of dynamic shared memory per CTA
-  for (warps = 8; warps >= 4; warps /= 2) {
-    const size_t per_warp = kBudget / warps;
-    const size_t fixed = kUpdownListCap * 8 + 128;
-    stages = per_warp > fixed ? static_cast<int>((per_warp - fixed) / (4 * static_cast<size_t>(K) + 8)) : 0;
-    if (stages > 8) stages = 8;
-    if (stages >= 2) return;
+  const size_t slot = 4 * static_cast<size_t>(K);
+  UpdownShape u{0, 0, 0};
+  if (max_warps >= 12) {
+    int cap = NT > C ? NT : C;
+    if (cap < 96) cap = 96;
+    cap = (cap + 31) / 32 * 32;
+    const size_t per_warp = kBudget / 12;
+    const size_t fixed = static_cast<size_t>(cap) * 8 + 128;
+    const int st = per_warp > fixed ? static_cast<int>((per_warp - fixed) / slot) : 0;
+    if (st >= 3) return {12, st > 8 ? 8 : st, cap};
   }
-  warps = 4;
+  for (int warps = 8; warps >= 4; warps /= 2) {
+    const size_t per_warp = kBudget / warps;
+    const size_t fixed = static_cast<size_t>(kUpdownListCap) * 8 + 128;
+    int st = per_warp > fixed ? static_cast<int>((per_warp - fixed) / slot) : 0;
+    if (st > 8) st = 8;
+    u = {warps, st, kUpdownListCap};
+    if (st >= 2) return u;
+  }
+  return u;
 }
 
 template <int KV>
 cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
                              float* y, int sms, cudaStream_t s) {
-  int warps = 8, stages = 2;
-  updown_config(tw->K, warps, stages);
-  if (stages < 1) return cudaErrorInvalidValue;
-  const size_t smem = static_cast<size_t>(warps) * updown_warp_bytes(tw->K, stages);
+  const UpdownShape u = updown_shape(tw->K, tw->N / tw->T, tw->C, updown_max_warps<KV>());
+  if (u.stages < 2) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(u.warps) * updown_warp_bytes(tw->K, u.stages, u.list_cap);
   cudaError_t e = cudaFuncSetAttribute(twell_updown_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -210,8 +227,9 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
   p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals;
   p.M = tw->M; p.K = tw->K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
   p.y = y; p.ctrl = tw->ctrl; p.units = reinterpret_cast<int4*>(tw->units);
-  p.stages = stages;
-  return launch_pdl(twell_updown_kernel<KV>, sms, 32 * warps, smem, s, p);
+  p.stages = u.stages;
+  p.list_cap = u.list_cap;
+  return launch_pdl(twell_updown_kernel<KV>, sms, 32 * u.warps, smem, s, p);
 }
 
 cudaError_t launch_updown(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw, float* y,

@@ -70,7 +70,8 @@ typedef enum {
  *   slot_row   int32  [R_cap]     row that owns each slot (valid for slots < n_over)
  *   ctrl       int32  [64]        device control words: [0] n_over (rows that
  *                                 asked for a slot), [1] status flags, [2..6]
- *                                 work-queue counters of the fused kernel
+ *                                 work-queue counters of the fused kernel, [7]
+ *                                 entries of the non-overflow tiles
  *   x_over     bf16   [R_cap][K]  scratch: gathered x rows of slotted rows
  *   h_over     bf16   [R_cap][2N] scratch: overflow-tile hidden activations as
  *                                 bf16 hi (columns < N) + lo (columns >= N) parts
