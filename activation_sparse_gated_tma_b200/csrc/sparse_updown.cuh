@@ -448,11 +448,17 @@ __global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_k
     ok = __shfl_sync(0xffffffffu, ready, 0) != 0;
   }
   const int n_units = ok ? ld_acquire(ctrl + kCtrlUnitTail) : 0;
+  // Every unit is published by now: warp g takes unit g directly, later units
+  // come from the queue (numbered from the warp count on), so that the warps
+  // arriving together do not all contend for one counter.
+  const int n_warps = static_cast<int>(gridDim.x * (blockDim.x >> 5));
+  const int gw = static_cast<int>(blockIdx.x * (blockDim.x >> 5)) + warp;
+  bool first_unit = true;
   while (ok) {
     int ux = 0, uy = 0, uz = 0;
     int have = 0;
     if (lane == 0) {
-      const int h = atomicAdd(ctrl + kCtrlUnitHead, 1);
+      const int h = first_unit ? gw : n_warps + atomicAdd(ctrl + kCtrlUnitHead, 1);
       if (h < n_units) {
         const int4 u = p.units[h];
         ux = u.x;
@@ -462,7 +468,9 @@ __global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_k
       }
     }
     have = __shfl_sync(0xffffffffu, have, 0);
+    // No direct unit means fewer units than warps, so the queue is empty too.
     if (!have) break;
+    first_unit = false;
     const int row = __shfl_sync(0xffffffffu, ux, 0);
     const int tb = __shfl_sync(0xffffffffu, uy, 0);
     const int te = __shfl_sync(0xffffffffu, uz, 0);

@@ -135,7 +135,7 @@ twell_status tmap_bf16(const void* ptr, uint64_t inner, uint64_t outer, uint32_t
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, units, total;
+  size_t ctrl, counts, idx, vals, row_slot, slot_row, dense_rows, x_over, h_over, units, z, total;
 };
 
 bool shape_ok(int M, int K, int N, int T, int C, int R_cap) {
@@ -158,6 +158,7 @@ Layout layout(int M, int K, int N, int T, int C, int R_cap) {
   L.x_over = o; o = align256(o + size_t(R_cap) * K * 2);
   L.h_over = o; o = align256(o + size_t(R_cap) * N * 4);
   L.units = o; o = align256(o + size_t(M) * NT * 16);
+  L.z = o; o = align256(o + (M <= TWELL_SMALL_M ? size_t(M) * N * 4 : 0));
   L.total = o;
   return L;
 }
@@ -166,19 +167,91 @@ twell_status check_buf(const twell_buf* tw) {
   if (!tw) return fail(TWELL_ERR_INVALID, "twell_buf is NULL");
   if (!shape_ok(tw->M, tw->K, tw->N, tw->T, tw->C, tw->R_cap)) return fail(TWELL_ERR_INVALID, "twell_buf has invalid sizes");
   if (!tw->counts || !tw->idx || !tw->vals || !tw->dense_rows || !tw->row_slot || !tw->slot_row || !tw->ctrl ||
-      !tw->x_over || !tw->h_over || !tw->units)
+      !tw->x_over || !tw->h_over || !tw->units || (tw->M <= TWELL_SMALL_M && !tw->z))
     return fail(TWELL_ERR_INVALID, "twell_buf is not initialised");
   return TWELL_OK;
 }
 
 // ---------------------------------------------------------------- small kernels
 // Start of a gate pass: no row holds a dense-row slot, control words at zero.
-__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl) {
+// The small-M path also clears z (n4 float4), which its split-K GEMM adds into.
+__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl,
+                                   float4* __restrict__ z, int64_t n4) {
   griddep_launch_dependents();
   griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < kCtrlWords) ctrl[i] = 0;
   for (int r = i; r < M; r += gridDim.x * blockDim.x) row_slot[r] = kSlotFree;
+  for (int64_t k = i; k < n4; k += static_cast<int64_t>(gridDim.x) * blockDim.x) z[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Small-M path: ReLU + TwELL packing of the fp32 gate pre-activations z, one
+// warp per (row, TwELL tile).  Lane l holds columns [l*T/32, +T/32); the
+// packed entries keep ascending column order, the count is the true count,
+// and overflow tiles take a dense-row slot, exactly as in the gate GEMM's
+// epilogue (see EpiGateTwell).
+template <int T>
+__global__ void __launch_bounds__(256) twell_pack_kernel(const float* __restrict__ z, const GateTwellParams p, int M,
+                                                         int* ctrl) {
+  griddep_launch_dependents();
+  griddep_wait();
+  constexpr int V = T / 32;
+  const int lane = threadIdx.x & 31;
+  const int NT = p.N / T;
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (item >= static_cast<int64_t>(M) * NT) return;  // the whole warp leaves together
+  const int row = static_cast<int>(item / NT);
+  const int t = static_cast<int>(item - static_cast<int64_t>(row) * NT);
+  const float4* src = reinterpret_cast<const float4*>(z + static_cast<int64_t>(row) * p.N + t * T + lane * V);
+  float v[V];
+#pragma unroll
+  for (int q = 0; q < V / 4; ++q) {
+    const float4 a = src[q];
+    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+  }
+  int mine = 0;
+#pragma unroll
+  for (int j = 0; j < V; ++j) mine += v[j] > 0.f ? 1 : 0;
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+  const int64_t rec = static_cast<int64_t>(row) * NT + t;
+  int off = incl - mine;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    if (v[j] > 0.f) {
+      if (off < p.C) {
+        p.idx[rec * p.C + off] = static_cast<uint8_t>(lane * V + j);
+        p.vals[rec * p.C + off] = v[j];
+      }
+      ++off;
+    }
+  }
+  if (lane == 0) {
+    p.counts[rec] = static_cast<uint16_t>(cnt);
+    if (cnt > 0 && cnt <= p.C) atomicAdd(ctrl + kCtrlEntries, cnt);
+  }
+  if (cnt <= p.C) return;
+  int slot = -1;
+  bool fresh = false;
+  if (lane == 0) slot = acquire_row_slot(p.row_slot, p.slot_row, p.r_cap, row, ctrl, fresh);
+  slot = __shfl_sync(0xffffffffu, slot, 0);
+  fresh = __shfl_sync(0xffffffffu, fresh ? 1 : 0, 0) != 0;
+  if (fresh) {
+    const uint4* xs = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(row) * p.K);
+    uint4* xd = reinterpret_cast<uint4*>(p.x_over + static_cast<int64_t>(slot) * p.K);
+    for (int k = lane; k < p.K / 8; k += 32) xd[k] = xs[k];
+  }
+  if (slot >= 0) {
+    float4* dst = reinterpret_cast<float4*>(p.dense_rows + static_cast<int64_t>(slot) * p.N + t * T + lane * V);
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q)
+      dst[q] = make_float4(relu_f(v[4 * q]), relu_f(v[4 * q + 1]), relu_f(v[4 * q + 2]), relu_f(v[4 * q + 3]));
+  }
 }
 
 // Launch shape of the fused kernel.
@@ -325,6 +398,7 @@ twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int 
   tw->x_over = reinterpret_cast<uint16_t*>(b + L.x_over);
   tw->h_over = reinterpret_cast<uint16_t*>(b + L.h_over);
   tw->units = b + L.units;
+  tw->z = M <= TWELL_SMALL_M ? reinterpret_cast<float*>(b + L.z) : nullptr;
   tw->M = M; tw->K = K; tw->N = N; tw->T = T; tw->C = C; tw->R_cap = R_cap;
   return TWELL_OK;
 }
@@ -347,19 +421,44 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
   if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
   if ((st = tmap_bf16(wg_t, K, N, bn, tm_wg)) != TWELL_OK) return st;
 
-  const int rgrid = static_cast<int>((static_cast<int64_t>(M) + 255) / 256 < 1024 ? (M + 255) / 256 : 1024);
+  const bool small = tw->z != nullptr;
+  const int64_t z4 = small ? static_cast<int64_t>(M) * N / 4 : 0;
+  const int64_t rwork = (z4 > M ? z4 : M);
+  const int rgrid = static_cast<int>((rwork + 255) / 256 < 1024 ? (rwork + 255) / 256 : 1024);
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, stream, tw->row_slot, M, tw->ctrl));
+  TW_CUDA(launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, stream, tw->row_slot, M, tw->ctrl,
+                     reinterpret_cast<float4*>(tw->z), z4));
   TW_CUDA(trace_end(stream, "twell_reset"));
 
   GateTwellParams p;
   p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.dense_rows = tw->dense_rows;
   p.row_slot = tw->row_slot; p.slot_row = tw->slot_row; p.x = x; p.x_over = tw->x_over;
   p.N = N; p.K = K; p.C = tw->C; p.r_cap = tw->R_cap;
-  GemmGeom g{M, N, K, nullptr, kGateGroupM, 0, 1};
-  TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_gate_twell(tw->T, bn, tm_x, tm_wg, g, p, tw->ctrl, gemm_grid(M, N, bn, dev.sms), stream));
-  TW_CUDA(trace_end(stream, "gate_twell_gemm"));
+  if (small) {
+    // One 128-row tile: cut K so that the tiles cover the SMs, add the slices
+    // into z, then pack.
+    CUtensorMap tm_wg128;
+    if ((st = tmap_bf16(wg_t, K, N, 128, tm_wg128)) != TWELL_OK) return st;
+    const int ks = choose_k_splits(M, N, 128, K, dev.sms);
+    EpiStoreF32::Params pz{tw->z, N, N, 1};
+    GemmGeom gz{M, N, K, nullptr, kGateGroupM, 0, ks};
+    TW_CUDA(trace_begin(stream));
+    TW_CUDA(launch_gate_splitk(tm_x, tm_wg128, gz, pz, tw->ctrl, gemm_grid(M, N, 128, dev.sms, ks), stream));
+    TW_CUDA(trace_end(stream, "gate_splitk_gemm"));
+    const int64_t items = static_cast<int64_t>(M) * (N / tw->T);
+    const int pgrid = static_cast<int>((items + 7) / 8);
+    TW_CUDA(trace_begin(stream));
+    if (tw->T == 128)
+      TW_CUDA(launch_pdl(twell_pack_kernel<128>, pgrid, 256, 0, stream, tw->z, p, M, tw->ctrl));
+    else
+      TW_CUDA(launch_pdl(twell_pack_kernel<256>, pgrid, 256, 0, stream, tw->z, p, M, tw->ctrl));
+    TW_CUDA(trace_end(stream, "twell_pack"));
+  } else {
+    GemmGeom g{M, N, K, nullptr, kGateGroupM, 0, 1};
+    TW_CUDA(trace_begin(stream));
+    TW_CUDA(launch_gate_twell(tw->T, bn, tm_x, tm_wg, g, p, tw->ctrl, gemm_grid(M, N, bn, dev.sms), stream));
+    TW_CUDA(trace_end(stream, "gate_twell_gemm"));
+  }
 
   if (n_over_host) {
     int n_over = 0;

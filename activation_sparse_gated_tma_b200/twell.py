@@ -37,7 +37,7 @@ class CapacityError(TwellError):
 class _TwellBuf(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("counts", "idx", "vals", "dense_rows", "row_slot", "slot_row", "ctrl", "x_over", "h_over",
-                 "units")] + \
+                 "units", "z")] + \
                [(n, ctypes.c_int) for n in ("M", "K", "N", "T", "C", "R_cap")]
 
 

@@ -76,6 +76,8 @@ typedef enum {
  *   h_over     bf16   [R_cap][2N] scratch: overflow-tile hidden activations as
  *                                 bf16 hi (columns < N) + lo (columns >= N) parts
  *   units      int32  [M*NT][4]   scratch: work units of rows split across warps
+ *   z          fp32   [M][N]      scratch, only for M <= TWELL_SMALL_M (else NULL):
+ *                                 the gate pre-activation of the small-M path
  */
 typedef struct twell_buf {
   uint16_t* counts;
@@ -88,8 +90,14 @@ typedef struct twell_buf {
   uint16_t* x_over;
   uint16_t* h_over;
   void* units;
+  float* z;
   int M, K, N, T, C, R_cap;
 } twell_buf;
+
+/* Batches of at most this many rows take the small-M gate path: a split-K
+ * gate GEMM into the fp32 scratch z, then a separate TwELL packing kernel
+ * (one 128-row tile cannot occupy the GPU otherwise). */
+#define TWELL_SMALL_M 128
 
 /* Bytes of device memory twell_buf_init needs for these sizes (0 if invalid). */
 size_t twell_buf_bytes(int M, int K, int N, int T, int C, int R_cap);

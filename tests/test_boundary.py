@@ -49,7 +49,7 @@ def test_buf_init_layout_is_aligned_and_disjoint():
     NT = N // T
     spans = [("ctrl", 64 * 4), ("counts", M * NT * 2), ("idx", M * NT * C), ("vals", M * NT * C * 4),
              ("row_slot", M * 4), ("slot_row", R * 4), ("dense_rows", R * N * 4), ("x_over", R * K * 2),
-             ("h_over", R * N * 4), ("units", M * NT * 16)]
+             ("h_over", R * N * 4), ("units", M * NT * 16), ("z", M * N * 4)]  # z: M <= TWELL_SMALL_M
     ranges = []
     for name, size in spans:
         p = getattr(b, name)
@@ -63,6 +63,16 @@ def test_buf_init_layout_is_aligned_and_disjoint():
     assert L.twell_buf_init(ctypes.byref(b), base, nbytes - 1, M, K, N, T, C, R) == tw.ERR_INVALID
     assert L.twell_buf_init(ctypes.byref(b), base + 16, nbytes, M, K, N, T, C, R) == tw.ERR_INVALID
     assert b"aligned" in L.twell_last_error()
+
+
+def test_small_m_scratch_only_for_small_batches():
+    L = tw.lib()
+    b = tw._TwellBuf()
+    for M, has_z in ((128, True), (129, False)):
+        assert L.twell_buf_init(ctypes.byref(b), 1 << 32, L.twell_buf_bytes(M, 256, 1024, 128, 8, 8),
+                                M, 256, 1024, 128, 8, 8) == tw.OK
+        assert (b.z is not None) == has_z
+    assert L.twell_buf_bytes(128, 256, 1024, 128, 8, 8) - L.twell_buf_bytes(129, 256, 1024, 128, 8, 8) > 128 * 1024 * 4 - 4096
 
 
 def _fake_buf():

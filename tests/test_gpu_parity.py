@@ -185,3 +185,14 @@ def test_kernel_trace_brackets_every_launch():
     names = [n for n, _ in tr.times_ms()]
     assert names == ["twell_reset", "gate_twell_gemm", "twell_updown", "overflow_up_gemm", "overflow_down_gemm"]
     assert all(ms > 0 for _, ms in tr.times_ms())
+
+
+def test_small_batch_takes_the_split_k_gate_path():
+    # M <= TWELL_SMALL_M: split-K gate GEMM into the fp32 scratch, then the packing kernel.
+    w, d, dev = _workload("sweep_m64_k2048_n8192_p99")
+    t = tw.TwellBuffers(w.M, w.K, w.N, w.T, w.C)
+    with tw.KernelTrace(capacity=8) as tr:
+        tw.gate_pack(dev["x"], dev["wg_t"], t)
+    torch.cuda.synchronize()
+    assert [n for n, _ in tr.times_ms()] == ["twell_reset", "gate_splitk_gemm", "twell_pack"]
+    assert tw.last_launch_count() == 3
