@@ -50,11 +50,11 @@ struct UpdownParams {
   int list_cap;    // list entries per warp: >= N/T and >= C
 };
 
-// Warps per CTA: twelve for K <= 1536 (the state of a warp fits 170
-// registers), else eight.
+// Most warps per CTA: twelve for K <= 2048 (a warp's state then fits the 168
+// registers that twelve warps leave each thread without spilling), else eight.
 template <int KV>
 constexpr int updown_max_warps() {
-  return KV <= 6 ? 12 : 8;
+  return KV <= 8 ? 12 : 8;
 }
 
 // acc += h * d for 8 bf16 elements of d, as four packed fp32x2 FMAs (each lane

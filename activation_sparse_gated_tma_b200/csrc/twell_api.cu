@@ -259,21 +259,22 @@ struct UpdownShape {
   int warps, stages, list_cap;
 };
 
-// Twelve warps (K <= 1536) with a list just large enough (>= N/T, >= C, >= 96
-// entries) when each warp still gets three ring stages; else eight warps with
-// the full list when each gets two; else four.
+// Twelve warps (K <= 2048) with a list just large enough (>= N/T,
+// >= C, >= 96 entries) when each warp still gets enough ring stages (three up
+// to K = 1536, two above); else eight warps with the full list when each gets
+// two; else four.
 UpdownShape updown_shape(int K, int NT, int C, int max_warps) {
   constexpr size_t kBudget = 232448;  // 227 KB of dynamic shared memory per CTA
   const size_t slot = 4 * static_cast<size_t>(K);
   UpdownShape u{0, 0, 0};
-  if (max_warps >= 12) {
+  if (max_warps > 8) {
     int cap = NT > C ? NT : C;
     if (cap < 96) cap = 96;
     cap = (cap + 31) / 32 * 32;
-    const size_t per_warp = kBudget / 12;
+    const size_t per_warp = kBudget / max_warps;
     const size_t fixed = static_cast<size_t>(cap) * 8 + 128;
     const int st = per_warp > fixed ? static_cast<int>((per_warp - fixed) / slot) : 0;
-    if (st >= 3) return {12, st > 8 ? 8 : st, cap};
+    if (st >= (K <= 1536 ? 3 : 2)) return {max_warps, st > 8 ? 8 : st, cap};
   }
   for (int warps = 8; warps >= 4; warps /= 2) {
     const size_t per_warp = kBudget / warps;
