@@ -113,9 +113,13 @@ twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int 
                             int R_cap);
 
 /*
- * Gate GEMM + ReLU + TwELL pack + overflow routing (one launch after a small
- * reset kernel).  x [M][K], wg_t [N][K] device bf16.  M, K, N must equal the
- * buffer's.  Fills every array of `tw` described above.
+ * Gate GEMM + ReLU + TwELL pack + overflow routing ("Sparser, Faster, Lighter
+ * Transformer Language Models", §3-4 steps 1-5, §3-6, §4-3).  x [M][K], wg_t
+ * [N][K] device bf16.  M, K, N must equal the buffer's.  Fills every array of
+ * `tw` described above.  Launches: a small reset kernel, then one gate GEMM
+ * whose epilogue packs TwELL; for M <= TWELL_SMALL_M instead a split-K gate
+ * GEMM into z and a packing kernel (the same records, order and overflow
+ * routing).
  *
  * n_over_host: if NULL the call is fully asynchronous; the overflow count stays
  * on the device (ctrl[0]) and twell_read_status reports it later.  If not NULL
@@ -128,8 +132,9 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
                              int* n_over_host, cudaStream_t stream);
 
 /*
- * Fused sparse up + down projection over `tw` (filled by twell_gate_pack on the
- * same stream), then the dense-row path for overflow tiles.  wu_t, wd [N][K]
+ * Fused sparse up + down projection over `tw` ("Sparser, Faster, Lighter
+ * Transformer Language Models", §3-5; filled by twell_gate_pack on the same
+ * stream), then the dense-row path for overflow tiles (§3-6, §4-3).  wu_t, wd [N][K]
  * device bf16; y [M][K] device fp32, fully overwritten.  K must equal tw->K.
  * Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
  * -2 in row_slot miss their overflow tiles and twell_read_status returns
