@@ -1,5 +1,7 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
 same seeded inputs.  Rules in tests/parity.py."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -196,3 +198,21 @@ def test_small_batch_takes_the_split_k_gate_path():
     torch.cuda.synchronize()
     assert [n for n, _ in tr.times_ms()] == ["twell_reset", "gate_splitk_gemm", "twell_pack"]
     assert tw.last_launch_count() == 3
+
+
+def test_maximum_sizes_on_both_gate_paths():
+    # K = 4096 (the largest K: the fused kernel's four-warp shape) and N/T = 256
+    # (the largest tile count), on the gate GEMM's own packing (M = 130) and on
+    # the small-batch path (the first 64 rows).
+    w = wl.Workload("max_m130_k4096_n32768_p99", 130, 4096, 32768, 128, 8, 7, p_mean=0.01, r_cap=130)
+    d = wl.generate(w)
+    _CACHE.clear()
+    for M in (130, 64):
+        wm = dataclasses.replace(w, M=M)
+        dm = dict(d, x=d["x"][:M])
+        dev = {k: P.to_dev(dm[k]) for k in ("x", "wg_t", "wu_t", "wd")}
+        t, n_over, y = _run_sparse(dev, wm, R_cap=M)
+        stats = _compare(wm, dm, t, y, np.arange(M))
+        print("max sizes M", M, "n_over", n_over, stats)
+        del dev, t, y
+        torch.cuda.empty_cache()
