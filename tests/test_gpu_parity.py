@@ -98,6 +98,14 @@ def test_ragged_shapes_full_compare(M, T, C):
     _compare(w, d, t, y, rows, dense_y=tw.dense_ffn(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"]))
 
 
+@pytest.mark.parametrize("M", [33, 200])
+def test_smallest_k_full_compare(M):
+    # K = 64: one K block for every GEMM (both gate paths: M = 33 and 200).
+    w, d, dev = _small(M, 64, 512, 128, 4, None, seed=M + 5, R_cap=M)
+    t, n_over, y = _run_sparse(dev, w, R_cap=M)
+    _compare(w, d, t, y, np.arange(M), dense_y=tw.dense_ffn(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"]))
+
+
 def test_all_gates_off_gives_exact_zero():
     w, d, dev = _small(130, 128, 512, 128, 4, bias=1e4, seed=1)
     t, n_over, y = _run_sparse(dev, w)
