@@ -33,7 +33,7 @@
 namespace twell {
 
 constexpr int kUpdownListCap = 256;  // largest list of a warp (entries per segment; also the N/T limit)
-constexpr int kUnitCap = 16;         // largest target entries per unit of a split row
+constexpr int kUnitCap = 32;         // largest target entries per unit of a split row
 
 struct UpdownParams {
   const uint16_t* x;
@@ -373,10 +373,13 @@ __global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_k
   griddep_launch_dependents();
   griddep_wait();
 
-  // Units of about total entries / warps entries when that is below
-  // kUnitCap: with few rows, heavy rows are cut finer so that every warp
-  // streams; never below 2 entries, whose fixed cost would dominate.
-  int unit_cap = ld_acquire(ctrl + kCtrlEntries) / static_cast<int>(gridDim.x * (blockDim.x >> 5));
+  // Units of about two thirds of (total entries / warps) entries, between 2
+  // and kUnitCap: larger units when every warp has many entries (fewer fixed
+  // per-unit costs), smaller ones when it has few (no warp is left with a
+  // long last unit); measured best at 16 for 24 entries per warp and at 32
+  // for 130-380.
+  const int per_warp = ld_acquire(ctrl + kCtrlEntries) / static_cast<int>(gridDim.x * (blockDim.x >> 5));
+  int unit_cap = 2 * per_warp / 3;
   unit_cap = unit_cap < 2 ? 2 : (unit_cap > kUnitCap ? kUnitCap : unit_cap);
 
   uint4 xv[KV];
