@@ -168,19 +168,39 @@ struct EpiGateTwell : EpiNoPrepare {
 };
 
 // ---------------------------------------------------------------------------
+// h as an unevaluated sum of two bf16 numbers: hi = bf16(h), lo = bf16(h - hi),
+// so |h - hi - lo| <= 2^-9 |h - hi| <= 2^-18 |h| (about 16 significant bits)
+// while the next GEMM still runs on bf16 tensor cores, once over hi and once
+// over lo against the same weights.
+__device__ __forceinline__ void split_bf16x8(const float (&h)[8], uint4& hi, uint4& lo) {
+  uint32_t a[4], b[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    a[e] = pack_bf16x2(h[2 * e], h[2 * e + 1]);
+    b[e] = pack_bf16x2(h[2 * e] - __uint_as_float(a[e] << 16), h[2 * e + 1] - __uint_as_float(a[e] & 0xFFFF0000u));
+  }
+  hi = make_uint4(a[0], a[1], a[2], a[3]);
+  lo = make_uint4(b[0], b[1], b[2], b[3]);
+}
+
+// ---------------------------------------------------------------------------
 // Dense FFN first stage: accumulator 0 = x W_g tile, accumulator 1 = x W_u
-// tile (same columns).  Writes h = h_u * ReLU(h_g) as bf16 ("Sparser, Faster,
-// Lighter Transformer Language Models", §1-1).
+// tile (same columns).  Writes h = h_u * ReLU(h_g) ("Sparser, Faster, Lighter
+// Transformer Language Models", §1-1) either as bf16 hi + lo parts (h [M][2N]:
+// hi in columns [0, N), lo in [N, 2N)) or, with split == 0, rounded to one
+// bf16 (h [M][N], as a plain bf16 dense FFN keeps it).
 struct EpiGatedProduct : EpiNoPrepare {
   static constexpr int kScratchBytes = 0;
   struct Params {
-    uint16_t* h;  // [M][N] bf16
+    uint16_t* h;  // [M][2N] (split) or [M][N] bf16
     int N;
+    int split;
   };
   template <int BN>
   static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
                                              int nb, int, int*, void*, int, int) {
     const bool valid = row < m_rows;
+    const int64_t ld = p.split ? 2 * static_cast<int64_t>(p.N) : p.N;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       uint32_t g[32], u[32];
@@ -188,18 +208,16 @@ struct EpiGatedProduct : EpiNoPrepare {
       tmem_ld_32x32(taddr + BN + c * 32, u);
       tmem_wait_ld();
       if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(p.h + static_cast<int64_t>(row) * p.N + nb * BN + c * 32);
+        uint4* dst = reinterpret_cast<uint4*>(p.h + static_cast<int64_t>(row) * ld + nb * BN + c * 32);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           float h[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) h[e] = __uint_as_float(u[8 * v + e]) * relu_f(__uint_as_float(g[8 * v + e]));
-          uint4 o;
-          o.x = pack_bf16x2(h[0], h[1]);
-          o.y = pack_bf16x2(h[2], h[3]);
-          o.z = pack_bf16x2(h[4], h[5]);
-          o.w = pack_bf16x2(h[6], h[7]);
-          dst[v] = o;
+          uint4 hi, lo;
+          split_bf16x8(h, hi, lo);
+          dst[v] = hi;
+          if (p.split) dst[v + p.N / 8] = lo;
         }
       }
     }
@@ -311,15 +329,7 @@ struct EpiOverflowProduct {
           float h[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) h[e] = pre.ov ? __uint_as_float(u[8 * v + e]) * pre.g[c * 32 + 8 * v + e] : 0.f;
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hi[e] = pack_bf16x2(h[2 * e], h[2 * e + 1]);
-            lo[e] = pack_bf16x2(h[2 * e] - __uint_as_float(hi[e] << 16),
-                                h[2 * e + 1] - __uint_as_float(hi[e] & 0xFFFF0000u));
-          }
-          dst_hi[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          dst_lo[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          split_bf16x8(h, dst_hi[v], dst_lo[v]);
         }
       }
     }

@@ -20,9 +20,12 @@
 //     lanes in 16-byte pieces: lane l holds elements [(j*32 + l)*8, +8).
 //   * The warp lists the unit's active entries (n, g) from the TwELL records of
 //     its non-overflow tiles into shared memory.
-//   * Lane 0 streams the rows W_u^T[n] and W_d[n] of upcoming entries into a
-//     private shared-memory ring with 1-D bulk copies (cp.async.bulk, no
-//     multicast, one mbarrier per slot), several entries ahead.
+//   * The rows W_u^T[n] and W_d[n] of upcoming entries stream into the warp's
+//     shared-memory ring, several entries ahead, as 16-byte cp.async copies
+//     that every lane issues for itself: lane l copies, and later reads, only
+//     the pieces l, l + 32, ... of each row, so completion is tracked per lane
+//     with commit/wait groups (one group per ring slot) and no barrier or
+//     mbarrier is needed.
 //   * Per entry: u = x_m . W_u^T[n] (warp shuffle reduce), h = u * g,
 //     partial += h * W_d[n].
 // Overflow tiles (count > C) are skipped here; the dense-row path adds them.
@@ -48,6 +51,8 @@ struct UpdownParams {
   int4* units;     // [M * N/T] published units {row, tile begin, tile end, unused}
   int stages;
   int list_cap;    // list entries per warp: >= N/T and >= C
+  int scan_target;                   // rows the split-off units wait for (M; M + 1 only under fault injection)
+  unsigned long long wait_limit_ns;  // limit of that wait
 };
 
 // Most warps per CTA: twelve for K <= 2048 (a warp's state then fits the 168
@@ -440,8 +445,8 @@ __global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_k
     int ready = 1;
     if (lane == 0) {
       const unsigned long long t0 = global_ns();
-      while (ld_acquire(ctrl + kCtrlScanned) < p.M) {
-        if (global_ns() - t0 > kWaitLimitNs) {
+      while (ld_acquire(ctrl + kCtrlScanned) < p.scan_target) {
+        if (global_ns() - t0 > p.wait_limit_ns) {
           set_flag(ctrl, kFlagWaitTimeout);
           ready = 0;
           break;

@@ -19,6 +19,10 @@ namespace {
 
 thread_local char g_err[512] = "";
 thread_local int g_launches = 0;
+// One-shot fault injection (twell_test_expire_wait): the wait limit, in ns, of
+// the next fused-kernel launch on this thread, whose wait target is then made
+// unreachable; 0 = none.
+thread_local long long g_expire_wait_ns = 0;
 
 // Optional launch tracing: events[2i] / events[2i+1] bracket the i-th kernel.
 struct Trace {
@@ -303,6 +307,13 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
   p.y = y; p.ctrl = tw->ctrl; p.units = reinterpret_cast<int4*>(tw->units);
   p.stages = u.stages;
   p.list_cap = u.list_cap;
+  p.scan_target = tw->M;
+  p.wait_limit_ns = kWaitLimitNs;
+  if (g_expire_wait_ns > 0) {
+    p.scan_target = tw->M + 1;
+    p.wait_limit_ns = static_cast<unsigned long long>(g_expire_wait_ns);
+    g_expire_wait_ns = 0;
+  }
   return launch_pdl(twell_updown_kernel<KV>, sms, 32 * u.warps, smem, s, p);
 }
 
@@ -338,6 +349,45 @@ int choose_k_splits(int rows, int cols, int bn, int K, int sms) {
   return (kb + per - 1) / per;
 }
 
+// Dense FFN ("Sparser, Faster, Lighter Transformer Language Models", §1-1
+// computed in full, §2-2 dense pipeline).  GEMM 1 puts x W_g and x W_u of the
+// same column tile into two TMEM accumulators and writes h; GEMM 2 computes
+// y = h W_d.  With `split`, h is stored as bf16 hi + lo halves (h [M][2N]) and
+// GEMM 2 reduces over [h_hi | h_lo] against W_d twice (b_k_wrap), so h keeps
+// about 16 significant bits; without it h is one bf16 (h [M][N]).
+twell_status dense_ffn_impl(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd, int M,
+                            int K, int N, uint16_t* h_scratch, float* y, bool split, cudaStream_t stream) {
+  g_launches = 0;
+  if (M < 1 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0)
+    return fail(TWELL_ERR_INVALID, "invalid sizes M=%d K=%d N=%d (need K %% 64 == 0, N %% 128 == 0)", M, K, N);
+  if (!aligned16(x) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(h_scratch) || !aligned16(y))
+    return fail(TWELL_ERR_INVALID, "all pointers must be non-NULL and 16-byte aligned");
+  twell_status st;
+  DeviceInfo dev;
+  if ((st = device_info(dev)) != TWELL_OK) return st;
+  const int hcols = split ? 2 * N : N;
+  CUtensorMap tm_x, tm_wg, tm_wu, tm_h, tm_wd;
+  if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wg_t, K, N, 128, tm_wg)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wu_t, K, N, 128, tm_wu)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(h_scratch, hcols, M, kBM, tm_h)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wd, K, N, 64, tm_wd)) != TWELL_OK) return st;
+
+  EpiGatedProduct::Params p1{h_scratch, N, split ? 1 : 0};
+  GemmGeom g1{M, N, K, nullptr, kGateGroupM, 0, 1};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_gated_product(tm_x, tm_wg, tm_wu, g1, p1, nullptr, gemm_grid(M, N, 128, dev.sms), stream));
+  TW_CUDA(trace_end(stream, "dense_gate_up_gemm"));
+  const int ks2 = choose_k_splits(M, K, 256, hcols, dev.sms);
+  if (ks2 > 1) TW_CUDA(cudaMemsetAsync(y, 0, static_cast<size_t>(M) * K * sizeof(float), stream));
+  EpiStoreF32::Params p2{y, K, K, ks2 > 1 ? 1 : 0};
+  GemmGeom g2{M, K, hcols, nullptr, kGateGroupM, split ? N / kBK : 0, ks2};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_down_store(tm_h, tm_wd, g2, p2, nullptr, gemm_grid(M, K, 256, dev.sms, ks2), stream));
+  TW_CUDA(trace_end(stream, "dense_down_gemm"));
+  return TWELL_OK;
+}
+
 }  // namespace
 }  // namespace twell
 
@@ -360,6 +410,13 @@ const char* twell_status_str(twell_status st) {
 const char* twell_last_error(void) { return g_err; }
 
 int twell_last_launch_count(void) { return g_launches; }
+
+twell_status twell_test_expire_wait(long long limit_ns) {
+  if (limit_ns != 0 && (limit_ns < 1000 || limit_ns > 1000000000))
+    return fail(TWELL_ERR_INVALID, "limit_ns must be 0 or in [1000, 1000000000], got %lld", limit_ns);
+  g_expire_wait_ns = limit_ns;
+  return TWELL_OK;
+}
 
 twell_status twell_trace_events(cudaEvent_t* events, int capacity) {
   if (events && capacity < 1) return fail(TWELL_ERR_INVALID, "capacity must be >= 1");
@@ -535,34 +592,12 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
 
 twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd, int M,
                            int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream) {
-  g_launches = 0;
-  if (M < 1 || K < 64 || K % 64 != 0 || N < 128 || N % 128 != 0)
-    return fail(TWELL_ERR_INVALID, "invalid sizes M=%d K=%d N=%d (need K %% 64 == 0, N %% 128 == 0)", M, K, N);
-  if (!aligned16(x) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(h_scratch) || !aligned16(y))
-    return fail(TWELL_ERR_INVALID, "all pointers must be non-NULL and 16-byte aligned");
-  twell_status st;
-  DeviceInfo dev;
-  if ((st = device_info(dev)) != TWELL_OK) return st;
-  CUtensorMap tm_x, tm_wg, tm_wu, tm_h, tm_wd;
-  if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(wg_t, K, N, 128, tm_wg)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(wu_t, K, N, 128, tm_wu)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(h_scratch, N, M, kBM, tm_h)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(wd, K, N, 64, tm_wd)) != TWELL_OK) return st;
+  return dense_ffn_impl(x, wg_t, wu_t, wd, M, K, N, h_scratch, y, true, stream);
+}
 
-  EpiGatedProduct::Params p1{h_scratch, N};
-  GemmGeom g1{M, N, K, nullptr, kGateGroupM, 0, 1};
-  TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_gated_product(tm_x, tm_wg, tm_wu, g1, p1, nullptr, gemm_grid(M, N, 128, dev.sms), stream));
-  TW_CUDA(trace_end(stream, "dense_gate_up_gemm"));
-  const int ks2 = choose_k_splits(M, K, 256, N, dev.sms);
-  if (ks2 > 1) TW_CUDA(cudaMemsetAsync(y, 0, static_cast<size_t>(M) * K * sizeof(float), stream));
-  EpiStoreF32::Params p2{y, K, K, ks2 > 1 ? 1 : 0};
-  GemmGeom g2{M, K, N, nullptr, kGateGroupM, 0, ks2};
-  TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_down_store(tm_h, tm_wd, g2, p2, nullptr, gemm_grid(M, K, 256, dev.sms, ks2), stream));
-  TW_CUDA(trace_end(stream, "dense_down_gemm"));
-  return TWELL_OK;
+twell_status dense_ffn_fwd_bf16h(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
+                                 int M, int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream) {
+  return dense_ffn_impl(x, wg_t, wu_t, wd, M, K, N, h_scratch, y, false, stream);
 }
 
 }  // extern "C"
@@ -570,32 +605,61 @@ twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16
 // ---------------------------------------------------------------------------
 // Dense FFN for callers that cannot allocate device memory at call time: a
 // runtime that has handed all device memory to its own pool, or an embedding
-// that forbids allocation while it executes.  The hidden activations h, which
-// dense_ffn_fwd takes as a caller buffer, live here in a fixed array that is
-// part of the library's device image; every device that loads the library
-// keeps it (32 MiB) until the process exits.
+// that forbids allocation while it executes.  The hidden activations h (bf16
+// hi + lo halves, [M][2N]), which dense_ffn_fwd takes as a caller buffer, live
+// here in a fixed array that is part of the library's device image; every
+// device that loads the library keeps it (32 MiB) until the process exits.
 namespace twell {
 namespace {
 
 constexpr size_t kNoAllocHiddenElems = size_t(16) << 20;  // 16 Mi bf16 values = 32 MiB
 __device__ __align__(256) uint16_t g_noalloc_hidden[kNoAllocHiddenElems];
 
-// Device address of the fixed array on the current device.  In host code the
-// array's name is only a host-side handle, so the address is looked up once per
-// device (with that device current) and cached.
-twell_status noalloc_hidden_ptr(uint16_t** out) {
-  int dev = 0;
-  TW_CUDA(cudaGetDevice(&dev));
-  static std::mutex mu;
-  static std::map<int, uint16_t*> addr;
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = addr.find(dev);
-  if (it == addr.end()) {
+// Id of the calling thread's current CUDA context (false if none is current
+// or the driver lacks the query).  Ids are never reused within a process, so
+// a context re-created after cudaDeviceReset gets a new one.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    TW_CUDA(cudaGetSymbolAddress(&p, g_noalloc_hidden));
-    it = addr.emplace(dev, static_cast<uint16_t*>(p)).first;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the fixed array in the current context.  In host code the
+// array's name is only a host-side handle, so the address is looked up with
+// cudaGetSymbolAddress (with the device current) and cached per context: a
+// context torn down by cudaDeviceReset and created again gets a new id, so the
+// address is looked up again rather than reused.
+twell_status noalloc_hidden_ptr(uint16_t** out) {
+  static std::mutex mu;
+  static std::map<unsigned long long, uint16_t*> addr;
+  unsigned long long ctx = 0;
+  bool have_ctx = current_context_id(&ctx);
+  std::lock_guard<std::mutex> lock(mu);
+  if (have_ctx) {
+    auto it = addr.find(ctx);
+    if (it != addr.end()) {
+      *out = it->second;
+      return TWELL_OK;
+    }
   }
-  *out = it->second;
+  void* p = nullptr;
+  TW_CUDA(cudaGetSymbolAddress(&p, g_noalloc_hidden));  // also makes the primary context current
+  if (!have_ctx) have_ctx = current_context_id(&ctx);
+  if (have_ctx) addr[ctx] = static_cast<uint16_t*>(p);
+  *out = static_cast<uint16_t*>(p);
   return TWELL_OK;
 }
 
@@ -606,10 +670,11 @@ extern "C" twell_status dense_ffn_fwd_noalloc(const uint16_t* x, const uint16_t*
                                               const uint16_t* wd, int M, int K, int N, float* y,
                                               cudaStream_t stream) {
   g_launches = 0;
-  if (M < 1 || N < 1 || static_cast<size_t>(M) * static_cast<size_t>(N) > kNoAllocHiddenElems)
+  if (M < 1 || N < 1 || 2 * static_cast<size_t>(M) * static_cast<size_t>(N) > kNoAllocHiddenElems)
     return fail(TWELL_ERR_INVALID,
-                "dense_ffn_fwd_noalloc: M*N = %lld exceeds the built-in scratch of %zu elements (32 MiB of bf16)",
-                static_cast<long long>(M) * N, kNoAllocHiddenElems);
+                "dense_ffn_fwd_noalloc: h needs M*2N = %lld bf16 values, more than the built-in scratch of %zu "
+                "(32 MiB)",
+                2 * static_cast<long long>(M) * N, kNoAllocHiddenElems);
   uint16_t* h = nullptr;
   twell_status st = noalloc_hidden_ptr(&h);
   if (st != TWELL_OK) return st;

@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
         "twell_ffn_fwd": (I, [P, P, P, BP, I, P, P]),
         "twell_read_status": (I, [BP, IP, IP, P]),
         "dense_ffn_fwd": (I, [P, P, P, P, I, I, I, P, P, P]),
+        "dense_ffn_fwd_bf16h": (I, [P, P, P, P, I, I, I, P, P, P]),
+        "dense_ffn_fwd_noalloc": (I, [P, P, P, P, I, I, I, P, P]),
+        "twell_test_expire_wait": (I, [ctypes.c_longlong]),
         "twell_status_str": (ctypes.c_char_p, [I]),
         "twell_last_error": (ctypes.c_char_p, []),
         "twell_last_launch_count": (I, []),
@@ -256,19 +259,47 @@ def read_status(tw: TwellBuffers, stream=None):
 
 
 def dense_ffn(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd: torch.Tensor,
-              h_scratch: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """dense_ffn_fwd: the same y with dense tensor-core GEMMs (h materialised in bf16)."""
+              h_scratch: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None, stream=None,
+              bf16_h: bool = False) -> torch.Tensor:
+    """dense_ffn_fwd: the same y with dense tensor-core GEMMs.
+
+    h is materialised as bf16 hi + lo halves (h_scratch [M][2N]); with
+    bf16_h=True, dense_ffn_fwd_bf16h keeps it as one bf16 (h_scratch [M][N]).
+    """
     M, K = x.shape
     N = wg_t.shape[0]
+    hcols = N if bf16_h else 2 * N
     if h_scratch is None:
-        h_scratch = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        h_scratch = torch.empty((M, hcols), dtype=torch.bfloat16, device=x.device)
     if y is None:
         y = torch.empty((M, K), dtype=torch.float32, device=x.device)
-    st = lib().dense_ffn_fwd(_bf16(x, "x", (M, K)), _bf16(wg_t, "wg_t", (N, K)), _bf16(wu_t, "wu_t", (N, K)),
-                             _bf16(wd, "wd", (N, K)), M, K, N, _bf16(h_scratch, "h_scratch", (M, N)), y.data_ptr(),
-                             _stream(stream))
-    _check(st, "dense_ffn_fwd")
+    if y.dtype != torch.float32 or not y.is_contiguous() or tuple(y.shape) != (M, K):
+        raise ValueError("y must be a contiguous float32 tensor of shape (M, K)")
+    f = lib().dense_ffn_fwd_bf16h if bf16_h else lib().dense_ffn_fwd
+    st = f(_bf16(x, "x", (M, K)), _bf16(wg_t, "wg_t", (N, K)), _bf16(wu_t, "wu_t", (N, K)),
+           _bf16(wd, "wd", (N, K)), M, K, N, _bf16(h_scratch, "h_scratch", (M, hcols)), y.data_ptr(),
+           _stream(stream))
+    _check(st, "dense_ffn_fwd_bf16h" if bf16_h else "dense_ffn_fwd")
     return y
+
+
+def dense_ffn_noalloc(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd: torch.Tensor,
+                      y: torch.Tensor, stream=None) -> torch.Tensor:
+    """dense_ffn_fwd_noalloc: dense_ffn with h in the library's fixed device array."""
+    M, K = x.shape
+    N = wg_t.shape[0]
+    if y.dtype != torch.float32 or not y.is_contiguous() or tuple(y.shape) != (M, K) or not y.is_cuda:
+        raise ValueError("y must be a contiguous CUDA float32 tensor of shape (M, K)")
+    st = lib().dense_ffn_fwd_noalloc(_bf16(x, "x", (M, K)), _bf16(wg_t, "wg_t", (N, K)),
+                                     _bf16(wu_t, "wu_t", (N, K)), _bf16(wd, "wd", (N, K)), M, K, N,
+                                     y.data_ptr(), _stream(stream))
+    _check(st, "dense_ffn_fwd_noalloc")
+    return y
+
+
+def test_expire_wait(limit_ns: int) -> None:
+    """twell_test_expire_wait: arm a one-shot expiring device wait for the next ffn_fwd."""
+    _check(lib().twell_test_expire_wait(int(limit_ns)), "twell_test_expire_wait")
 
 
 def sparse_ffn(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd: torch.Tensor, T: int, C: int,

@@ -99,8 +99,8 @@ WORKLOADS: Dict[str, Workload] = {
          for j, p in enumerate([0.1, 0.01, 0.001])]
 }
 
-#: The single-GPU throughput workload (99% sparsity, per-token counts varying ~10x).
-BENCH_WORKLOAD = "m2048_k1536_n4096_p99_lognormal05"
+#: The single-GPU throughput workload: the largest configuration at 99% sparsity.
+BENCH_WORKLOAD = "m16384_k2560_n10240_p99_boost3pct"
 #: The small case the oracle finishes in seconds.
 TINY_WORKLOAD = "tiny_m64_k256_n1024_p98"
 PARITY_WORKLOADS: List[str] = [

@@ -1,14 +1,20 @@
 """Throughput of the sparse gated FFN forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload NAME] [--no-cpu-baseline]
+                    [--workload NAME] [--no-cpu-baseline] [--no-extra]
 
 One step = one pass of the whole sparse path over one batch of M tokens:
 twell_gate_pack (reset + tcgen05 gate GEMM with the ReLU/TwELL/overflow
-epilogue) followed by twell_ffn_fwd (fused sparse up+down kernel, then the
-dense-row overflow GEMMs), asynchronous, inputs resident in HBM.  The L2
-(126 MB) is flushed with a 256 MiB write before every timed step; the flush
-is outside the timed events.
+epilogue), twell_ffn_fwd (fused sparse up+down kernel, then the dense-row
+overflow GEMMs) and one device-to-host read of the overflow count and the
+device flags, which the host checks after the step (a count above the
+dense-row capacity would make the caller retry with a larger buffer), inputs
+resident in HBM.  The L2 (126 MB) is flushed with a 256 MiB write before
+every timed step; the flush is outside the timed events.
+
+The headline workload is the largest single-GPU configuration at 99%
+sparsity (M=16384, K=2560, N=10240); the M=2048 and M=8192 workloads are
+timed the same way and reported under "other_workloads".
 
 For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
 same workload: the forward pass is token-parallel and needs no collective
@@ -43,6 +49,8 @@ UNIT = "tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILES = os.path.join(ROOT, "profiles")
+# Timed next to the headline workload and reported under "other_workloads".
+EXTRA_WORKLOADS = ("m2048_k1536_n4096_p99_lognormal05", "m8192_k2048_n5632_loguniform_lognormal07")
 FLUSH_BYTES = 256 << 20
 
 
@@ -249,17 +257,40 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- native arm
-def run_native(args, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
-    from activation_sparse_gated_tma_b200 import twell as tw
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = wl.WORKLOADS[args.workload]
-    d = wl.generate(w)
+def path_roofline(M, K, N, T, C, U, R, peaks, ms):
+    """The path roofline as the scope table's measurement rule states it:
+    T_roof = max(2MKN / P_tc, B_alg / BW_hbm) with
+    B_alg = 2KN + 4K*U + 2MK + 4MK + 2*M*(N/T)*(2+3C) + 4*R*N
+    (W_g once; the unique W_u, W_d rows; x; y in fp32; TwELL written and read
+    with bf16 values; the bf16 dense-row backup written and read)."""
+    NT = N // T
+    flops = 2.0 * M * K * N
+    b_alg = 2.0 * K * N + 4.0 * K * U + 2.0 * M * K + 4.0 * M * K + 2.0 * M * NT * (2 + 3 * C) + 4.0 * R * N
+    # This build stores TwELL values and the dense-row gates in fp32: 5 bytes per slot, 4 per gate.
+    b_build = 2.0 * K * N + 4.0 * K * U + 2.0 * M * K + 4.0 * M * K + 2.0 * M * NT * (2 + 5 * C) + 8.0 * R * N
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = b_alg / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_tc, t_hbm)
+    return {"t_roof_ms": t_roof * 1e3, "t_step_ms": ms, "frac": t_roof * 1e3 / ms,
+            "bound": "tensor" if t_tc >= t_hbm else "hbm",
+            "flops": flops, "bytes": b_alg, "P_tc_tflops": peaks["bf16_tflops"], "BW_hbm_gbs": peaks["hbm_gbs"],
+            "U": U, "R": R, "bytes_fp32_vals_variant": b_build,
+            "frac_fp32_vals_variant": max(t_tc, b_build / (peaks["hbm_gbs"] * 1e9)) * 1e3 / ms}
 
+
+def measure_workload(tw, torch, dev, w, d, steps, warmup, flush, peaks, peak_kind, clocks=None, full=True):
+    """Time one workload: the sparse step three ways, each kernel, both dense FFNs."""
     def to_dev(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
 
@@ -267,55 +298,81 @@ def run_native(args, rank, world, local_rank):
     M, K, N, T, C = w.M, w.K, w.N, w.T, w.C
     tb = tw.TwellBuffers(M, K, N, T, C, device=dev)
     y = torch.empty(M, K, dtype=torch.float32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    words = torch.zeros(2, dtype=torch.int32).pin_memory()
+    ctrl = tb.ctrl
 
-    def step():
+    launches = [0]
+
+    def step_async():
         tw.gate_pack(x, wg, tb)
         n1 = tw.last_launch_count()
         tw.ffn_fwd(x, wu, wd, tb, y)
-        return n1 + tw.last_launch_count()
+        launches[0] += n1 + tw.last_launch_count()
+
+    def step_read_status():
+        # The whole step, then one D2H of the overflow count and the device flags
+        # (checked on the host once the step's end event has completed).
+        step_async()
+        words.copy_(ctrl[:2], non_blocking=True)
+
+    def check_words():
+        n_over, flags = int(words[0]), int(words[1])
+        if flags != 0 or n_over > tb.R_cap:
+            raise RuntimeError(f"{w.name}: device flags 0x{flags:x}, n_over {n_over} (R_cap {tb.R_cap})")
+        return n_over
+
+    def step_sync_gate():
+        tw.gate_pack(x, wg, tb, sync=True)      # syncs, reads n_over, checks capacity
+        n1 = tw.last_launch_count()
+        tw.ffn_fwd(x, wu, wd, tb, y)
+        launches[0] += n1 + tw.last_launch_count()
+
+    def timed(fn, after=None):
+        out = []
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            if after:
+                after()
+            out.append(a.elapsed_time(b))
+        return sum(out) / len(out)
 
     # Correctness of the configuration before timing: capacity and device flags.
-    step()
-    st, n_over, flags = tw.read_status(tb)
+    step_read_status()
+    torch.cuda.synchronize()
+    n_over = check_words()
+    st, _, _ = tw.read_status(tb)
     if st != tw.OK:
-        raise RuntimeError(f"sparse path status {st} (n_over={n_over}, flags={flags}); raise R_cap")
+        raise RuntimeError(f"{w.name}: sparse path status {st}")
     stats = workload_stats(tb, w, T, C)
     U = unique_active_units(tb, C, T)
 
-    for _ in range(args.warmup):
-        step()
+    for _ in range(warmup):
+        step_read_status()
     torch.cuda.synchronize()
+    launches[0] = 0
+    if clocks is not None:
+        with clocks:
+            ms = timed(step_read_status, check_words)
+    else:
+        ms = timed(step_read_status, check_words)
+    n_launches = launches[0]
+    ms_async = timed(step_async)
+    ms_sync = timed(step_sync_gate)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    launches = 0
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            starts[i].record()
-            launches += step()
-            ends[i].record()
-        torch.cuda.synchronize()
-        barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(step_ms) / len(step_ms)
-
-    # Per-kernel durations: the same K steps again with an event pair around
+    # Per-kernel durations: the same steps again with an event pair around
     # every kernel (events between kernels stop a launch from overlapping the
     # previous kernel's tail, so these steps are not the ones timed above).
     traces = []
-    for i in range(args.steps):
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         tr = tw.KernelTrace(capacity=8)
         with tr:
-            step()
+            step_async()
         traces.append(tr)
     torch.cuda.synchronize()
     per_kernel = {}
@@ -324,32 +381,102 @@ def run_native(args, rank, world, local_rank):
             per_kernel.setdefault(name, []).append(t)
     kern_ms = {k: sum(v) / len(v) for k, v in per_kernel.items()}
 
+    # The in-build dense tcgen05 FFN on the same inputs (same flush discipline):
+    # h as bf16 hi + lo (held to the same accuracy rule as the sparse path), and
+    # the plain bf16-h variant as a second, labelled number.
+    h = torch.empty(M, 2 * N, dtype=torch.bfloat16, device=dev)
+    yd = torch.empty(M, K, dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        tw.dense_ffn(x, wg, wu, wd, h, yd)
+    dense_ms = timed(lambda: tw.dense_ffn(x, wg, wu, wd, h, yd))
+    h1 = h.view(-1)[:M * N].view(M, N)
+    for _ in range(warmup):
+        tw.dense_ffn(x, wg, wu, wd, h1, yd, bf16_h=True)
+    dense_bf16h_ms = timed(lambda: tw.dense_ffn(x, wg, wu, wd, h1, yd, bf16_h=True))
+    del h, h1, yd
 
-    # In-build dense tcgen05 FFN on the same inputs (same flush discipline).
-    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    for _ in range(args.warmup):
-        tw.dense_ffn(x, wg, wu, wd, h, y)
-    dense_ms = []
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        tw.dense_ffn(x, wg, wu, wd, h, y)
-        b.record()
-        b.synchronize()
-        dense_ms.append(a.elapsed_time(b))
-    dense_ms = sum(dense_ms) / len(dense_ms)
+    NT = N // T
+    flops_gate = 2.0 * M * K * N
+    entries = stats["twell_entries"]
+    bytes_updown = (2.0 * M * K                      # x rows
+                    + 2.0 * M * NT                   # counts
+                    + 5.0 * entries                  # idx + fp32 value per listed entry
+                    + 4.0 * K * U                    # unique W_u^T and W_d rows
+                    + 4.0 * M * K)                   # y (fp32)
+    kernels = {}
+    for name, t in kern_ms.items():
+        if name == "gate_twell_gemm":
+            ach = flops_gate / (t * 1e-3) / 1e12
+            kernels[name] = {"ms": t, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                             "algorithmic": flops_gate}
+        elif name == "twell_updown":
+            ach = bytes_updown / (t * 1e-3) / 1e9
+            kernels[name] = {"ms": t, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": ach / peaks["hbm_gbs"], "algorithmic": bytes_updown,
+                             "l2_gather_gbs": 4.0 * K * entries / (t * 1e-3) / 1e9}
+        elif name in ("overflow_up_gemm", "overflow_down_gemm"):
+            # dense-equivalent work of the slotted rows: one K x N product each
+            # (the down GEMM runs it twice, over the hi and lo halves of h)
+            f = 2.0 * n_over * K * N * (2 if name == "overflow_down_gemm" else 1)
+            kernels[name] = {"ms": t, "bound": "tensor", "achieved": f / (t * 1e-3) / 1e12, "unit": "TFLOP/s",
+                             "peak": peaks["bf16_tflops"], "frac": f / (t * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                             "algorithmic": f}
+        else:
+            kernels[name] = {"ms": t}
+    dominant = max(kern_ms.items(), key=lambda kv: kv[1])[0]
+    dom = kernels[dominant]
+    roofline = {"kernel": dominant, "bound": dom.get("bound"), "achieved": dom.get("achieved"),
+                "peak": dom.get("peak"), "unit": dom.get("unit"), "frac": dom.get("frac"),
+                "traffic": profiled_traffic(dominant, w.name), "peak_source": peak_kind + " (burst)"}
+    out = {
+        "workload": w.name, "M": M, "K": K, "N": N, "T": T, "C": C, "R_cap": tb.R_cap,
+        "ms_per_step": ms, "value": M / (ms * 1e-3),
+        "ms_per_step_async": ms_async, "ms_per_step_sync_gate": ms_sync,
+        "sparsity": stats, "unique_units_gathered": U, "n_over": n_over,
+        "roofline": roofline, "path_roofline": path_roofline(M, K, N, T, C, U, n_over, peaks, ms),
+        "kernels": kernels,
+        "dense": {"ms_per_step": dense_ms, "value": M / (dense_ms * 1e-3), "unit": UNIT,
+                  "variant": "dense_ffn_fwd: h as bf16 hi + lo, held to the same y rule as the sparse path"},
+        "dense_bf16h": {"ms_per_step": dense_bf16h_ms, "value": M / (dense_bf16h_ms * 1e-3), "unit": UNIT,
+                        "variant": "dense_ffn_fwd_bf16h: h rounded to one bf16 (not held to the y rule)"},
+        "speedup_vs_dense": dense_ms / ms, "speedup_vs_dense_bf16h": dense_bf16h_ms / ms,
+        "gpu_launches": n_launches,
+    }
+    out["_tensors"] = (x, wg, wu, wd, tb, y)
+    return out
 
-    # End to end through the public API with host buffers: pinned x in, y out.
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from activation_sparse_gated_tma_b200 import twell as tw
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    w = wl.WORKLOADS[args.workload]
+    d = wl.generate(w)
+    clk = ClockSampler(local_rank)
+    head = measure_workload(tw, torch, dev, w, d, args.steps, args.warmup, flush, peaks, peak_kind, clocks=clk)
+    x, wg, wu, wd, tb, y = head.pop("_tensors")
+
+    # End to end through the public API with host buffers: pinned x in, y out,
+    # plus the overflow count and device flags (twell_read_status).
     x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    y_host = torch.empty(M, K, dtype=torch.float32).pin_memory()
+    y_host = torch.empty(w.M, w.K, dtype=torch.float32).pin_memory()
     x_e2e = torch.empty_like(x)
+    words = torch.zeros(2, dtype=torch.int32).pin_memory()
 
     def e2e_step():
         x_e2e.copy_(x_host, non_blocking=True)
         tw.gate_pack(x_e2e, wg, tb)
         tw.ffn_fwd(x_e2e, wu, wd, tb, y)
         y_host.copy_(y, non_blocking=True)
+        words.copy_(tb.ctrl[:2], non_blocking=True)
 
     for _ in range(args.warmup):
         e2e_step()
@@ -361,76 +488,62 @@ def run_native(args, rank, world, local_rank):
         e2e_step()
         b.record()
         b.synchronize()
+        if int(words[1]) != 0 or int(words[0]) > tb.R_cap:
+            raise RuntimeError(f"end-to-end step: device flags {int(words[1])}, n_over {int(words[0])}")
         e2e_ms.append(a.elapsed_time(b))
     e2e_ms = sum(e2e_ms) / len(e2e_ms)
+    del x, wg, wu, wd, tb, y, x_e2e
+
+    # The other full-size workloads, measured the same way (same steps).
+    others = {}
+    if not args.no_extra:
+        for name in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            wo = wl.WORKLOADS[name]
+            r = measure_workload(tw, torch, dev, wo, wl.generate(wo), args.steps, args.warmup, flush, peaks,
+                                 peak_kind)
+            r.pop("_tensors")
+            others[name] = r
+            torch.cuda.empty_cache()
 
     # One collective on every rank: the job's time is the slowest rank's.
-    ms, dense_ms, e2e_ms = max_over_ranks([ms, dense_ms, e2e_ms], world, dev)
+    ms, e2e_ms = max_over_ranks([head["ms_per_step"], e2e_ms], world, dev)
     if rank != 0:
         return
-
-    peaks, peak_kind = load_peaks()
-    # Algorithmic quantities per launch / per step.
-    flops_gate = 2.0 * M * K * N
-    NT = N // T
-    bytes_updown = (2.0 * M * K                      # x rows
-                    + 2.0 * M * NT                   # counts
-                    + 5.0 * stats["twell_entries"]   # idx + fp32 value per listed entry
-                    + 4.0 * K * U                    # unique W_u^T and W_d rows
-                    + 4.0 * M * K)                   # y (fp32)
-    R = n_over
-    flops_over = 2.0 * R * K * N * 2                 # up and down GEMMs of the slotted rows
-    bytes_path = (2.0 * K * N + 4.0 * K * U + 2.0 * M * K + 4.0 * M * K + 2.0 * M * NT * (2 + 5 * C)
-                  + 8.0 * R * N)
-    t_roof_s = max((flops_gate + flops_over) / (peaks["bf16_tflops"] * 1e12), bytes_path / (peaks["hbm_gbs"] * 1e9))
-    kernels = {}
-    for name, t in kern_ms.items():
-        if name == "gate_twell_gemm":
-            ach = flops_gate / (t * 1e-3) / 1e12
-            kernels[name] = {"ms": t, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
-        elif name == "twell_updown":
-            ach = bytes_updown / (t * 1e-3) / 1e9
-            kernels[name] = {"ms": t, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": ach / peaks["hbm_gbs"],
-                             "l2_gather_gbs": 4.0 * K * stats["twell_entries"] / (t * 1e-3) / 1e9}
-        else:
-            kernels[name] = {"ms": t}
-    dominant = max(kern_ms.items(), key=lambda kv: kv[1])[0]
-    dom = kernels[dominant]
-    roofline = {"kernel": dominant, "bound": dom.get("bound"), "achieved": dom.get("achieved"),
-                "peak": dom.get("peak"), "unit": dom.get("unit"), "frac": dom.get("frac"),
-                "traffic": profiled_traffic(dominant, w.name), "peak_source": peak_kind + " (burst)"}
 
     cpu = None
     if not args.no_cpu_baseline:
         rate, rows, sec, cores = cpu_oracle_rate(d, w, rows_target_s=12.0)
-        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
                "sample": f"{rows} seeded rows of {w.M} ({sec:.1f} s): fp64 gate, TwELL pack, sparse y"}
 
-    value = job_throughput(world, M, ms)
+    value = job_throughput(world, w.M, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "C": C, "R_cap": w.R_cap,
-                   "global_batch": world * M, "parallelism": f"replicas{world}",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "T": w.T, "C": w.C, "R_cap": head["R_cap"],
+                   "global_batch": world * w.M, "parallelism": f"replicas{world}",
                    "l2": "flushed: 256 MiB write before each timed step (outside the timed events)",
-                   "mode": "asynchronous gate_pack (overflow count stays on the device)"},
-        "sparsity": stats, "unique_units_gathered": U,
-        "roofline": roofline,
-        "path_roofline": {"t_roof_ms": t_roof_s * 1e3, "frac": t_roof_s * 1e3 / ms,
-                          "bound": "tensor" if (flops_gate + flops_over) / (peaks["bf16_tflops"] * 1e12)
-                          >= bytes_path / (peaks["hbm_gbs"] * 1e9) else "hbm",
-                          "flops": flops_gate + flops_over, "bytes": bytes_path},
-        "kernels": kernels,
-        "dense": {"ms_per_step": dense_ms, "value": job_throughput(world, M, dense_ms), "unit": UNIT},
-        "speedup_vs_dense": dense_ms / ms,
+                   "mode": "step = twell_gate_pack + twell_ffn_fwd + one D2H of the overflow count and device "
+                           "flags, checked on the host after the step (capacity retry on overflow)"},
+        "ms_per_step_async": head["ms_per_step_async"], "ms_per_step_sync_gate": head["ms_per_step_sync_gate"],
+        "sparsity": head["sparsity"], "unique_units_gathered": head["unique_units_gathered"],
+        "n_over": head["n_over"],
+        "roofline": head["roofline"],
+        "path_roofline": path_roofline(w.M, w.K, w.N, w.T, w.C, head["unique_units_gathered"], head["n_over"],
+                                       peaks, ms),
+        "kernels": head["kernels"],
+        "dense": head["dense"], "dense_bf16h": head["dense_bf16h"],
+        "speedup_vs_dense": head["dense"]["ms_per_step"] / ms,
+        "speedup_vs_dense_bf16h": head["dense_bf16h"]["ms_per_step"] / ms,
         "cpu_baseline": cpu,
-        "e2e": {"value": job_throughput(world, M, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * M * K,
-                "d2h_bytes_per_step": 4 * M * K, "ms_per_step": e2e_ms},
-        "gpu_launches": launches,
+        "e2e": {"value": job_throughput(world, w.M, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": 2 * w.M * w.K,
+                "d2h_bytes_per_step": 4 * w.M * w.K + 8, "ms_per_step": e2e_ms},
+        "gpu_launches": head["gpu_launches"],
         "clocks": clk.summary(),
+        "other_workloads": others,
     }
     print(json.dumps(line), flush=True)
 
@@ -443,6 +556,7 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default=wl.BENCH_WORKLOAD, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time only --workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -154,12 +154,26 @@ twell_status twell_read_status(const twell_buf* tw, int* n_over_host, int* devic
 /*
  * Dense comparison FFN (§1-1 computed in full, §2-2 "dense pipeline"):
  * GEMM 1 computes x W_g and x W_u for the same column tile into two TMEM
- * accumulators and writes h = (x W_u) * ReLU(x W_g) as bf16 into h_scratch
- * [M][N] (device, caller-owned); GEMM 2 writes y = h W_d, fp32 [M][K].
- * Limits: K % 64 == 0, N % 128 == 0.  Asynchronous.
+ * accumulators and writes h = (x W_u) * ReLU(x W_g) into h_scratch as two
+ * bf16 halves, hi = bf16(h) in columns [0, N) and lo = bf16(h - hi) in
+ * columns [N, 2N) of h_scratch [M][2N] (device, caller-owned); GEMM 2 writes
+ * y = h_hi W_d + h_lo W_d, fp32 [M][K].  h keeps about 16 significant bits, so
+ * y meets the same accuracy bound as the sparse path (a single bf16 h leaves
+ * an error of 2^-9 of each row's own scale, which heavy-tailed rows carry far
+ * above the global rms of y).  Limits: K % 64 == 0, N % 128 == 0.
+ * Asynchronous.
  */
 twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
                            int M, int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream);
+
+/*
+ * The same dense FFN with h rounded to a single bf16 (h_scratch [M][N]), as a
+ * plain bf16 dense FFN keeps it.  Faster than dense_ffn_fwd (GEMM 2 reduces
+ * over N, not 2N) but less accurate: reported next to it as a second dense
+ * comparison point, not held to the sparse path's accuracy bound.
+ */
+twell_status dense_ffn_fwd_bf16h(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
+                                 int M, int K, int N, uint16_t* h_scratch, float* y, cudaStream_t stream);
 
 /*
  * dense_ffn_fwd without a caller-provided hidden buffer, for callers that
@@ -168,19 +182,35 @@ twell_status dense_ffn_fwd(const uint16_t* x, const uint16_t* wg_t, const uint16
  * it executes).  The pages describe no such variant; it is an interface
  * convenience of this library.
  *
- * The hidden activations use a fixed 32 MiB array inside the library's device
- * image (every device that loads the library holds it until the process exits),
- * so M * N must not exceed 16,777,216; larger problems return
- * TWELL_ERR_INVALID with a message and launch nothing.  No device memory is
- * allocated or freed by this call.  The first call on a device looks up the
- * array's device address (with that device current); make that first call
- * before any stream capture.  All calls share the one array and it keeps the
- * last call's contents, so calls that overlap on the GPU (other streams, other
- * host threads) race on it; serialise them.  Otherwise identical to
- * dense_ffn_fwd: y [M][K] fp32 is overwritten, asynchronous on `stream`.
+ * The hidden activations (bf16 hi + lo, M x 2N values) use a fixed 32 MiB
+ * array inside the library's device image (every device that loads the
+ * library holds it until the process exits), so M * 2N must not exceed
+ * 16,777,216 (M * N <= 8,388,608); larger problems return TWELL_ERR_INVALID
+ * with a message and launch nothing.  No device memory is allocated or freed
+ * by this call.  The array's device address is looked up with
+ * cudaGetSymbolAddress on the first call in each CUDA context (with that
+ * context's device current) and cached per context id, so a context that
+ * cudaDeviceReset tore down and the runtime created again is looked up anew;
+ * make the first call in a context before any stream capture.  All calls share
+ * the one array and it keeps the last call's contents, so calls that overlap
+ * on the GPU (other streams, other host threads) race on it; serialise them.
+ * Otherwise identical to dense_ffn_fwd: y [M][K] fp32 is overwritten,
+ * asynchronous on `stream`.
  */
 twell_status dense_ffn_fwd_noalloc(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
                                    int M, int K, int N, float* y, cudaStream_t stream);
+
+/*
+ * Host-side fault injection for tests of the device status path.  Arms a
+ * one-shot for the next twell_ffn_fwd on this thread: its fused kernel waits
+ * for one more scanned token row than exist, a condition nothing makes true,
+ * with a wait limit of limit_ns nanoseconds instead of the usual 2 s.  The
+ * wait expires, the kernel raises its timeout flag and returns (the rows of
+ * split work units are then left incomplete), and twell_read_status reports
+ * TWELL_ERR_DEVICE_CHECK.  The next twell_gate_pack clears the flag.  No
+ * memory access changes.  limit_ns must lie in [1000, 1000000000]; 0 disarms.
+ */
+twell_status twell_test_expire_wait(long long limit_ns);
 
 /* Static description of a status code. */
 const char* twell_status_str(twell_status status);

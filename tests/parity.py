@@ -16,13 +16,17 @@ stated targets and the arithmetic of each side):
     room for the tensor core's internal alignment of partial sums).
   * Overflow classification equals the oracle's unless ambiguous entries
     straddle C (then both count sides stay within the ambiguous range).
-  * y (sparse path, fp32 intermediates): max |y_gpu - y64| <= 2e-2 * rms(y64)
-    over all compared entries.
-  * y (dense comparison path, h rounded to bf16 like a bf16 dense FFN): the
-    same bound per token row, max_k |y_gpu - y64| <= 2e-2 * rms_k(y64[m]),
-    with rms_k floored at 1e-3 of the global rms.  bf16 h carries a relative
-    error of 2^-9 of each row's own scale, and with heavy-tailed token scales
-    the largest rows sit 20-50x above the global rms.
+  * y (sparse path and dense_ffn_fwd, both with fp32 or hi+lo bf16
+    intermediates): max |y_gpu - y64| <= 2e-2 * rms(y64) over all compared
+    entries, rms taken over the whole compared block.
+  * y of the bf16-h dense variant (dense_ffn_fwd_bf16h, reported next to the
+    dense path but not held to the rule above): elementwise
+    |y_gpu - y64| <= sum_n dh[m,n] |W_d[n,k]| + N * 2^-23 * A + 1e-6 * rms(y64)
+    with A[m,k] = sum_n |h64[m,n]| |W_d[n,k]| and the error of the stored h
+    dh = 2^-9 |h64| + K * 2^-22 * (S_u |g64| + S_g |u64|): rounding h to bf16
+    (relative error <= 2^-9) plus the fp32 accumulation of u and g (the values
+    rule above, S_u and S_g the absolute-product sums of each); then the fp32
+    accumulation of N products in the second GEMM.
 """
 from __future__ import annotations
 
@@ -119,14 +123,20 @@ def check_y(y_gpu: np.ndarray, y64: np.ndarray, what: str = "y") -> dict:
     return {"rms": rms, "max_err": err, "rel": err / rms}
 
 
-def check_y_rows(y_gpu: np.ndarray, y64: np.ndarray, what: str = "y") -> dict:
-    g_rms = float(np.sqrt((y64 ** 2).mean()))
-    r_rms = np.sqrt((y64 ** 2).mean(1))
-    err = np.abs(y_gpu.astype(np.float64) - y64).max(1)
-    tol = Y_REL_TOL * np.maximum(r_rms, 1e-3 * g_rms)
-    zero = r_rms == 0.0
-    assert (err[zero] == 0.0).all(), f"{what}: rows with exact-zero output differ"
-    worst = float((err[~zero] / tol[~zero]).max()) if (~zero).any() else 0.0
-    assert worst <= 1.0, f"{what}: per-row error {worst:.3g} x tolerance"
-    return {"rms": g_rms, "max_err": float(err.max()), "rel_global": float(err.max() / g_rms) if g_rms else 0.0,
-            "row_err_over_tol": worst}
+def check_y_bf16h(y_gpu: np.ndarray, y64: np.ndarray, u64: np.ndarray, z64: np.ndarray, S_u: np.ndarray,
+                  S_g: np.ndarray, wd_bits: np.ndarray, K: int, what: str = "bf16-h dense y") -> dict:
+    """Elementwise bound for the dense variant that rounds h to one bf16."""
+    g64 = np.maximum(z64, 0.0)
+    h64 = u64 * g64
+    # S_g |u| also covers units the fp32 gate turns on where z64 <= 0 (then g_gpu <= K 2^-22 S_g)
+    dh = 2.0 ** -9 * np.abs(h64) + K * 2.0 ** -22 * (S_u * g64 + S_g * np.abs(u64))
+    wd = np.abs(bf16_f64(wd_bits))
+    N = wd.shape[0]
+    tol = dh @ wd + N * 2.0 ** -23 * (np.abs(h64) @ wd)
+    rms = float(np.sqrt((y64 ** 2).mean()))
+    tol += 1e-6 * rms
+    err = np.abs(y_gpu.astype(np.float64) - y64)
+    worst = float((err / tol).max())
+    assert worst <= 1.0, f"{what}: error {worst:.3g} x the bf16-h bound"
+    return {"rms": rms, "max_err": float(err.max()), "rel": float(err.max() / rms) if rms else 0.0,
+            "err_over_bound": worst}

@@ -105,6 +105,23 @@ def test_ffn_fwd_and_dense_validate_before_launch():
     assert L.dense_ffn_fwd(p, p, p, p, 64, 200, 1024, p, p, None) == tw.ERR_INVALID      # K % 64
     assert L.dense_ffn_fwd(p, p, p, p, 64, 256, 1000, p, p, None) == tw.ERR_INVALID      # N % 128
     assert L.dense_ffn_fwd(p, p, p, p, 64, 256, 1024, None, p, None) == tw.ERR_INVALID
+    assert L.dense_ffn_fwd_bf16h(p, p, p, p, 64, 256, 1000, p, p, None) == tw.ERR_INVALID
+
+
+def test_expire_wait_hook_validates_its_limit():
+    L = tw.lib()
+    assert L.twell_test_expire_wait(10) == tw.ERR_INVALID
+    assert L.twell_test_expire_wait(2_000_000_000) == tw.ERR_INVALID
+    assert L.twell_test_expire_wait(5000) == tw.OK
+    assert L.twell_test_expire_wait(0) == tw.OK       # disarm: nothing launched here
+
+
+def test_noalloc_rejects_oversize_before_any_cuda_call():
+    L = tw.lib()
+    p = 1 << 33
+    # h needs M * 2N bf16 values; the fixed array holds 16 Mi.
+    assert L.dense_ffn_fwd_noalloc(p, p, p, p, 2049, 256, 4096, p, None) == tw.ERR_INVALID
+    assert b"built-in scratch" in L.twell_last_error()
 
 
 def test_python_wrapper_rejects_wrong_tensors():
