@@ -16,8 +16,9 @@
 //     (the first one too) then adds its partial y_m with vector atomics, so no
 //     warp ever waits for another.
 // Inside a unit:
-//   * x_m (bf16) and the fp32 partial of y_m stay in registers, spread over the
-//     lanes in 16-byte pieces: lane l holds elements [(j*32 + l)*8, +8).
+//   * x_m (bf16, read with an L2 evict-first hint) and the fp32 partial of y_m
+//     stay in registers, spread over the lanes in 16-byte pieces: lane l holds
+//     elements [(j*32 + l)*8, +8).
 //   * The warp lists the unit's active entries (n, g) from the TwELL records of
 //     its non-overflow tiles into shared memory.
 //   * The rows W_u^T[n] and W_d[n] of upcoming entries stream into the warp's
@@ -292,6 +293,19 @@ __device__ __forceinline__ void stream_entries(const UpdownParams& p, const Warp
   }
 }
 
+// 16-byte read-only load with an L2 evict-first hint: x rows are read once per
+// row or unit, while the gathered weight rows (evict-last) are reused across
+// rows and should keep their place in L2.
+__device__ __forceinline__ uint4 ldg_evict_first(const uint4* src) {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(src), "l"(pol));
+  return v;
+}
+
 template <int KV>
 __device__ __forceinline__ void load_x(const UpdownParams& p, int row, uint4 (&xv)[KV], float (&acc)[KV][8],
                                        int lane) {
@@ -299,7 +313,7 @@ __device__ __forceinline__ void load_x(const UpdownParams& p, int row, uint4 (&x
 #pragma unroll
   for (int j = 0; j < KV; ++j) {
     const int k0 = (j * 32 + lane) * 8;
-    xv[j] = k0 < p.K ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
+    xv[j] = k0 < p.K ? ldg_evict_first(reinterpret_cast<const uint4*>(xr + k0)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
   }
