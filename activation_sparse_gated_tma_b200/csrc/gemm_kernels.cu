@@ -30,6 +30,31 @@ cudaError_t launch_gate_twell(int T, int bn, const CUtensorMap& tm_x, const CUte
   return cudaErrorInvalidValue;
 }
 
+namespace {
+template <int T>
+cudaError_t launch_pair_t(const CUtensorMap& a, const CUtensorMap& b, const GemmGeom& g, const GateTwellParams& p,
+                          int* ctrl, int grid, cudaStream_t s) {
+  using Epi = EpiGateTwell<T>;
+  constexpr int warps = Epi::template kWarps<256>;
+  constexpr int kStages = gemm_pair_smem_bytes<6, Epi::kScratchBytes, warps>() <= 232448 ? 6 : 5;
+  constexpr size_t smem = gemm_pair_smem_bytes<kStages, Epi::kScratchBytes, warps>();
+  static_assert(smem <= 232448, "exceeds the 227 KB per-CTA shared memory limit");
+  auto kern = tc_gemm_pair_kernel<kStages, Epi>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if (grid <= 0) return cudaSuccess;
+  return launch_pdl_pair(kern, grid, gemm_threads<Epi, 256>(), smem, s, a, b, g, p, ctrl);
+}
+}  // namespace
+
+cudaError_t launch_gate_twell_pair(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
+                                   const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s) {
+  if (grid % 2) return cudaErrorInvalidValue;
+  if (T == 128) return launch_pair_t<128>(tm_x, tm_wg, g, p, ctrl, grid, s);
+  if (T == 256) return launch_pair_t<256>(tm_x, tm_wg, g, p, ctrl, grid, s);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_gate_splitk(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
                                const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s) {
   return launch<128, false, false, 6, EpiStoreF32>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);

@@ -17,6 +17,10 @@ namespace twell {
 // CTA tile width bn in {128, 256}, a multiple of T.
 cudaError_t launch_gate_twell(int T, int bn, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
                               const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s);
+// Gate GEMM on CTA pairs (cta_group::2, 256 x 256 tiles; see tc_gemm_pair_kernel):
+// tm_wg's box is 128 rows (each CTA's half of a tile's columns).  grid is even.
+cudaError_t launch_gate_twell_pair(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
+                                   const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s);
 // Small-M gate: z += x W_g (fp32, vector atomics per K slice), BN = 128.
 cudaError_t launch_gate_splitk(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
                                const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s);
@@ -52,6 +56,27 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// launch_pdl for clusters of two CTAs.
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl_pair(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 

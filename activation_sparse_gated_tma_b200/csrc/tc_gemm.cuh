@@ -241,4 +241,161 @@ __global__ void __launch_bounds__(gemm_threads<Epi, BN>(), 1)
   if (warp == 1) tmem_dealloc(tmem_base, L::kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// Two-CTA variant for K-major A and B: a cluster of two CTAs (one per SM)
+// computes each 256 x 256 tile with cta_group::2 UMMA (M = 256).  Rank r loads
+// its own 128 rows of A and its own 128 columns of B (no multicast): the pair
+// moves 2/3 of the operand bytes per FLOP of a one-CTA 128 x 256 tile, which
+// matters because the one-CTA engine is bound by the L2 -> SM operand rate,
+// not by the tensor pipe.  Both CTAs' loads complete on the leader's (rank 0)
+// full barrier; the leader's single MMA thread issues the UMMAs and its
+// commits reach the empty / accumulator-full barriers of both CTAs.  Each CTA's
+// epilogue reads its own TMEM (its 128 rows, all 256 columns) and arrives on
+// the leader's accumulator-empty barrier.
+template <int STAGES, int EPI_SCRATCH, int EPI_WARPS>
+constexpr size_t gemm_pair_smem_bytes() {
+  return 1024 + static_cast<size_t>(STAGES) * 2 * kBM * kBK * 2 + (2 * STAGES + 4) * sizeof(uint64_t) + 16 + 128 +
+         EPI_WARPS * static_cast<size_t>(EPI_SCRATCH);
+}
+
+template <int STAGES, class Epi>
+__global__ void __launch_bounds__(gemm_threads<Epi, 256>(), 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const GemmGeom g, const typename Epi::Params ep, int* ctrl) {
+  constexpr int BN = 256;                   // tile columns (both CTAs); each CTA holds BN / 2 of B
+  constexpr int kABytes = kBM * kBK * 2;    // this CTA's 128 rows of A
+  constexpr int kBBytes = kBM * kBK * 2;    // this CTA's 128 columns of B
+  constexpr int kStageBytes = kABytes + kBBytes;
+  constexpr uint32_t kAccCols = BN;
+  constexpr uint32_t kTmemCols = 2 * kAccCols;
+  constexpr int kEpiWarps = Epi::template kWarps<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint8_t* epi_scratch = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tmem_holder + 4) + 127) & ~uintptr_t(127));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // used in the leader: its producer's expect_tx + both CTAs' bytes
+      mbar_init(&empty[s], 1);  // both CTAs: the leader's commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);                   // both CTAs: the leader's commit
+      mbar_init(&tempty[a], 2 * 32 * kEpiWarps);  // used in the leader: both CTAs' epilogue threads
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before any arrival reaches them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  griddep_launch_dependents();
+  griddep_wait();
+
+  int m_rows = g.M;
+  if (g.m_limit) m_rows = min(m_rows, *g.m_limit);
+  const int num_m = (m_rows + 2 * kBM - 1) / (2 * kBM);
+  const int num_n = (g.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int total_kb = g.K / kBK;
+  const int cluster = static_cast<int>(blockIdx.x >> 1);
+  const int nclusters = static_cast<int>(gridDim.x >> 1);
+
+  if (warp == 0) {
+    if (lane == 0 && num_tiles > cluster) {
+      prefetch_tmap(&tmA);
+      prefetch_tmap(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < num_tiles && ok; tile += nclusters) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, g.group_m, mb, nb);
+        for (int kb = 0; kb < total_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, ctrl)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          const uint32_t bar = mapa_shared(&full[stage], 0);
+          uint8_t* sa = smem + stage * kStageBytes;
+          tma_load_2d_pair(&tmA, bar, sa, kb * kBK, mb * 2 * kBM + static_cast<int>(rank) * kBM);
+          tma_load_2d_pair(&tmB, bar, sa + kABytes, kb * kBK, nb * BN + static_cast<int>(rank) * kBM);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, BN, false, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < num_tiles && ok; tile += nclusters, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, ctrl)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * kAccCols;
+        for (int kb = 0; kb < total_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, ctrl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k)
+            umma_bf16_pair(d, smem_desc_sw128(a_base + k * 32, 16, 1024), smem_desc_sw128(b_base + k * 32, 16, 1024),
+                           idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_commit_pair(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) umma_commit_pair(&tfull[acc]);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    constexpr int kParts = kEpiWarps / 4;
+    const int part = (warp - 2) >> 2;
+    const uint32_t tempty_leader0 = mapa_shared(&tempty[0], 0);
+    const uint32_t tempty_leader1 = mapa_shared(&tempty[1], 0);
+    int it = 0;
+    for (int tile = cluster; tile < num_tiles; tile += nclusters, ++it) {
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, g.group_m, mb, nb);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      const int row = mb * 2 * kBM + static_cast<int>(rank) * kBM + row_in_tile;
+      typename Epi::template Pre<BN> pre;
+      Epi::template prepare<BN>(ep, pre, row, m_rows, nb);
+      if (!mbar_wait(&tfull[acc], acc_phase, ctrl)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kAccCols;
+      Epi::template run<BN>(ep, pre, taddr, row, m_rows, nb, lane, ctrl,
+                            epi_scratch + (warp - 2) * Epi::kScratchBytes, part, kParts);
+      tc_fence_before();
+      mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still reach its shared memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
 }  // namespace twell

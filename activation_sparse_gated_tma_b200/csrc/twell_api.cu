@@ -511,6 +511,16 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
     else
       TW_CUDA(launch_pdl(twell_pack_kernel<256>, pgrid, 256, 0, stream, tw->z, p, M, tw->ctrl));
     TW_CUDA(trace_end(stream, "twell_pack"));
+  } else if (M > 256 && N % 256 == 0 && dev.sms >= 2) {
+    // CTA pairs on 256 x 256 tiles: each CTA moves 2/3 of the operand bytes per FLOP.
+    CUtensorMap tm_wg128;
+    if ((st = tmap_bf16(wg_t, K, N, 128, tm_wg128)) != TWELL_OK) return st;
+    const long tiles = static_cast<long>((M + 255) / 256) * (N / 256);
+    const int pairs = static_cast<int>(tiles < dev.sms / 2 ? tiles : dev.sms / 2);
+    GemmGeom g{M, N, K, nullptr, kGateGroupM / 2, 0, 1};
+    TW_CUDA(trace_begin(stream));
+    TW_CUDA(launch_gate_twell_pair(tw->T, tm_x, tm_wg128, g, p, tw->ctrl, 2 * pairs, stream));
+    TW_CUDA(trace_end(stream, "gate_twell_gemm"));
   } else {
     GemmGeom g{M, N, K, nullptr, kGateGroupM, 0, 1};
     TW_CUDA(trace_begin(stream));
