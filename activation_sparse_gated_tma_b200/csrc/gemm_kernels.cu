@@ -55,11 +55,6 @@ cudaError_t launch_gate_twell_pair(int T, const CUtensorMap& tm_x, const CUtenso
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_gate_splitk(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
-                               const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s) {
-  return launch<128, false, false, 6, EpiStoreF32>(tm_x, tm_wg, tm_wg, g, p, ctrl, grid, s);
-}
-
 cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
                                  const GemmGeom& g, const EpiGatedProduct::Params& p, int* ctrl, int grid,
                                  cudaStream_t s) {

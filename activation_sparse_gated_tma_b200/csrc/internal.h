@@ -21,9 +21,6 @@ cudaError_t launch_gate_twell(int T, int bn, const CUtensorMap& tm_x, const CUte
 // tm_wg's box is 128 rows (each CTA's half of a tile's columns).  grid is even.
 cudaError_t launch_gate_twell_pair(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
                                    const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s);
-// Small-M gate: z += x W_g (fp32, vector atomics per K slice), BN = 128.
-cudaError_t launch_gate_splitk(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
-                               const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s);
 // h = (x W_u) * ReLU(x W_g), bf16, BN = 128.
 cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
                                  const GemmGeom& g, const EpiGatedProduct::Params& p, int* ctrl, int grid,

@@ -29,6 +29,7 @@ enum : int {
   kCtrlUnitTail = 5,   //   split-off units published
   kCtrlScanned = 6,    //   rows whose units are all published
   kCtrlEntries = 7,    // TwELL entries listed by the gate pass (non-overflow tiles)
+  kCtrlGridSync = 8,   // single-kernel small-batch forward: CTAs past the gate phase
   kCtrlWords = 64,
 };
 
@@ -44,6 +45,14 @@ __device__ __forceinline__ unsigned long long global_ns() {
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
+
+// Acquire-release fence at GPU scope (lighter than __threadfence's sequentially
+// consistent one); pairs with a writer's fence before its flag update.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Orders this thread's shared-memory accesses in the generic proxy against
+// those of the async proxy (TMA writes, tensor-core reads) to the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void set_flag(int* ctrl, int flag) {
   if (ctrl) atomicOr(ctrl + kCtrlFlags, flag);
@@ -168,6 +177,20 @@ __device__ __forceinline__ void tmem_ld_32x32(uint32_t taddr, uint32_t (&r)[32])
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
       : "memory");
+}
+// 32 TMEM lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+// Barrier over `threads` threads (a multiple of 32) of the CTA, id 1..15.
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 

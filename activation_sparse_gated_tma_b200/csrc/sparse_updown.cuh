@@ -54,6 +54,10 @@ struct UpdownParams {
   int list_cap;    // list entries per warp: >= N/T and >= C
   int scan_target;                   // rows the split-off units wait for (M; M + 1 only under fault injection)
   unsigned long long wait_limit_ns;  // limit of that wait
+  // Small-batch kernel only (twell_updown_small_kernel):
+  const int* row_slot;      // [M] dense-row slot of each row (< 0: none)
+  const float* dense_rows;  // [R_cap][N] ReLU gates of overflow tiles
+  int tiles_per_unit;       // TwELL tiles per static work unit (1..32)
 };
 
 // Most warps per CTA: twelve for K <= 2048 (a warp's state then fits the 168
@@ -154,6 +158,7 @@ __device__ __forceinline__ int list_entries(const UpdownParams& p, const WarpRin
   const int NT = p.N / p.T;
   const uint16_t* crow = p.counts + static_cast<int64_t>(row) * NT;
   int E = 0;
+  __syncwarp();  // every lane is done reading the previous list
   while (cursor < te) {
     const int t = cursor + lane;
     const int c = t < te ? static_cast<int>(crow[t]) : 0;
@@ -522,6 +527,95 @@ __global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_k
       ctrl[kCtrlDone] = 0;
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Small batches (at most TWELL_SMALL_M rows).  With few rows the queue-based
+// kernel above leaves most warps idle or waiting on the row scan; here the
+// work is cut statically instead: unit u is row u / G of the tile group
+// u % G (tiles_per_unit consecutive TwELL tiles), and the warps take units
+// in turn (numbered warp-major across the CTAs).  A unit holds at most tiles_per_unit * C TwELL entries, so
+// every warp's chain is short, and no warp ever waits for another.  Overflow
+// tiles are served here too, from the row's dense-row slot (every positive
+// gate of the tile, in ascending order): small batches run no dense-row
+// GEMMs.  Every unit adds its partial y_m with vector atomics into y, which
+// the host clears first.  Weight rows used by several tokens of the batch are
+// read from HBM once and then from L2 (evict-last).
+// One warp's share of the small-batch units: units first, first + stride, ...
+template <int KV>
+__device__ __forceinline__ void run_small_units(const UpdownParams& p, const WarpRing& w, int64_t first, int64_t stride,
+                                                int lane) {
+  const int NT = p.N / p.T;
+  const int tpu = p.tiles_per_unit;
+  const int groups = (NT + tpu - 1) / tpu;
+  const int64_t n_units = static_cast<int64_t>(p.M) * groups;
+  uint4 xv[KV];
+  float acc[KV][8];
+  for (int64_t u = first; u < n_units; u += stride) {
+    const int row = static_cast<int>(u / groups);
+    const int t0 = static_cast<int>(u - static_cast<int64_t>(row) * groups) * tpu;
+    const int t1 = t0 + tpu < NT ? t0 + tpu : NT;
+    const int c = t0 + lane < t1 ? static_cast<int>(p.counts[static_cast<int64_t>(row) * NT + t0 + lane]) : 0;
+    if (__ballot_sync(0xffffffffu, c > 0) == 0) continue;
+    const uint32_t ov = __ballot_sync(0xffffffffu, c > p.C);
+    load_x<KV>(p, row, xv, acc, lane);
+    int cursor = t0;
+    while (cursor < t1) {
+      const int E = list_entries(p, w, row, cursor, t1, lane);
+      if (E > 0) stream_entries<KV>(p, w, E, xv, acc, lane);
+    }
+    const int slot = ov ? p.row_slot[row] : -1;
+    if (slot >= 0) {
+      uint32_t rest = ov;
+      int E = 0;
+      __syncwarp();
+      while (rest) {
+        const int t = t0 + __ffs(rest) - 1;
+        rest &= rest - 1;
+        if (E + p.T > w.list_cap) {
+          __syncwarp();
+          stream_entries<KV>(p, w, E, xv, acc, lane);
+          E = 0;
+          __syncwarp();
+        }
+        const float* src = p.dense_rows + static_cast<int64_t>(slot) * p.N + static_cast<int64_t>(t) * p.T;
+        for (int j0 = 0; j0 < p.T; j0 += 32) {
+          const float gv = src[j0 + lane];
+          const uint32_t bal = __ballot_sync(0xffffffffu, gv > 0.f);
+          if (gv > 0.f) {
+            const int pos = E + __popc(bal & ((1u << lane) - 1u));
+            w.list_n[pos] = t * p.T + j0 + lane;
+            w.list_g[pos] = gv;
+          }
+          E += __popc(bal);
+        }
+      }
+      __syncwarp();
+      if (E > 0) stream_entries<KV>(p, w, E, xv, acc, lane);
+    }
+    write_y<KV>(p, row, acc, true, lane);
+  }
+}
+
+template <int KV>
+__global__ void __launch_bounds__(32 * updown_max_warps<KV>(), 1) twell_updown_small_kernel(const UpdownParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  WarpRing w;
+  w.slot_bytes = 4u * p.K;
+  w.stages = p.stages;
+  w.ring = smem + static_cast<size_t>(warp) * updown_warp_bytes(p.K, p.stages, p.list_cap);
+  w.list_n = reinterpret_cast<int*>(w.ring + static_cast<size_t>(p.stages) * w.slot_bytes);
+  w.list_g = reinterpret_cast<float*>(w.list_n + p.list_cap);
+  w.list_cap = p.list_cap;
+  w.policy = l2_evict_last_policy();
+  griddep_launch_dependents();
+  griddep_wait();
+  // Consecutive units go to different SMs (warp-major numbering), so that a
+  // batch with fewer units than warps still spreads over every SM.
+  run_small_units<KV>(p, w, static_cast<int64_t>(warp) * gridDim.x + blockIdx.x,
+                      static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5), lane);
 }
 
 }  // namespace twell

@@ -12,7 +12,7 @@
 
 #include "../../include/twell.h"
 #include "internal.h"
-#include "sparse_updown.cuh"
+#include "fused_small.cuh"
 
 namespace twell {
 namespace {
@@ -162,7 +162,8 @@ Layout layout(int M, int K, int N, int T, int C, int R_cap) {
   L.x_over = o; o = align256(o + size_t(R_cap) * K * 2);
   L.h_over = o; o = align256(o + size_t(R_cap) * N * 4);
   L.units = o; o = align256(o + size_t(M) * NT * 16);
-  L.z = o; o = align256(o + (M <= TWELL_SMALL_M ? size_t(M) * N * 4 : 0));
+  // Small batches: partial gate sums [N/128][kStreamSlots][M][128] fp32, then one ticket per TwELL tile.
+  L.z = o; o = align256(o + (M <= TWELL_SMALL_M ? size_t(kStreamSlots) * M * N * 4 + NT * 4 : 0));
   L.total = o;
   return L;
 }
@@ -178,83 +179,131 @@ twell_status check_buf(const twell_buf* tw) {
 
 // ---------------------------------------------------------------- small kernels
 // Start of a gate pass: no row holds a dense-row slot, control words at zero.
-// The small-M path also clears z (n4 float4), which its split-K GEMM adds into.
-__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl,
-                                   float4* __restrict__ z, int64_t n4) {
+// The small-batch path also clears its n_tickets tile tickets.
+__global__ void twell_reset_kernel(int* __restrict__ row_slot, int M, int* __restrict__ ctrl, int* __restrict__ tickets,
+                                   int n_tickets) {
   griddep_launch_dependents();
   griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < kCtrlWords) ctrl[i] = 0;
   for (int r = i; r < M; r += gridDim.x * blockDim.x) row_slot[r] = kSlotFree;
-  for (int64_t k = i; k < n4; k += static_cast<int64_t>(gridDim.x) * blockDim.x) z[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = i; k < n_tickets; k += gridDim.x * blockDim.x) tickets[k] = 0;
 }
 
-// Small-M path: ReLU + TwELL packing of the fp32 gate pre-activations z, one
-// warp per (row, TwELL tile).  Lane l holds columns [l*T/32, +T/32); the
-// packed entries keep ascending column order, the count is the true count,
-// and overflow tiles take a dense-row slot, exactly as in the gate GEMM's
-// epilogue (see EpiGateTwell).
-template <int T>
-__global__ void __launch_bounds__(256) twell_pack_kernel(const float* __restrict__ z, const GateTwellParams p, int M,
-                                                         int* ctrl) {
-  griddep_launch_dependents();
-  griddep_wait();
-  constexpr int V = T / 32;
-  const int lane = threadIdx.x & 31;
-  const int NT = p.N / T;
-  const int64_t item = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (item >= static_cast<int64_t>(M) * NT) return;  // the whole warp leaves together
-  const int row = static_cast<int>(item / NT);
-  const int t = static_cast<int>(item - static_cast<int64_t>(row) * NT);
-  const float4* src = reinterpret_cast<const float4*>(z + static_cast<int64_t>(row) * p.N + t * T + lane * V);
-  float v[V];
-#pragma unroll
-  for (int q = 0; q < V / 4; ++q) {
-    const float4 a = src[q];
-    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
-  }
-  int mine = 0;
-#pragma unroll
-  for (int j = 0; j < V; ++j) mine += v[j] > 0.f ? 1 : 0;
-  int incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  const int cnt = __shfl_sync(0xffffffffu, incl, 31);
-  const int64_t rec = static_cast<int64_t>(row) * NT + t;
-  int off = incl - mine;
-#pragma unroll
-  for (int j = 0; j < V; ++j) {
-    if (v[j] > 0.f) {
-      if (off < p.C) {
-        p.idx[rec * p.C + off] = static_cast<uint8_t>(lane * V + j);
-        p.vals[rec * p.C + off] = v[j];
-      }
-      ++off;
-    }
-  }
-  if (lane == 0) {
-    p.counts[rec] = static_cast<uint16_t>(cnt);
-    if (cnt > 0 && cnt <= p.C) atomicAdd(ctrl + kCtrlEntries, cnt);
-  }
-  if (cnt <= p.C) return;
-  int slot = -1;
-  bool fresh = false;
-  if (lane == 0) slot = acquire_row_slot(p.row_slot, p.slot_row, p.r_cap, row, ctrl, fresh);
-  slot = __shfl_sync(0xffffffffu, slot, 0);
-  fresh = __shfl_sync(0xffffffffu, fresh ? 1 : 0, 0) != 0;
-  if (fresh) {
-    const uint4* xs = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(row) * p.K);
-    uint4* xd = reinterpret_cast<uint4*>(p.x_over + static_cast<int64_t>(slot) * p.K);
-    for (int k = lane; k < p.K / 8; k += 32) xd[k] = xs[k];
-  }
-  if (slot >= 0) {
-    float4* dst = reinterpret_cast<float4*>(p.dense_rows + static_cast<int64_t>(slot) * p.N + t * T + lane * V);
-#pragma unroll
-    for (int q = 0; q < V / 4; ++q)
-      dst[q] = make_float4(relu_f(v[4 * q]), relu_f(v[4 * q + 1]), relu_f(v[4 * q + 2]), relu_f(v[4 * q + 3]));
+// Tickets of the small-batch gate pass (after the partial sums in z).
+int* small_tickets(const twell_buf* tw) {
+  return reinterpret_cast<int*>(tw->z + static_cast<size_t>(kStreamSlots) * tw->M * tw->N);
+}
+
+// Operand ring depth of the small-batch gate pass in `budget` bytes of
+// shared memory (at most kStreamMaxStages).
+int stream_stages(int mp, size_t budget) {
+  const size_t fixed = 1024 + kStreamCtrlBytes;
+  const int st = budget > fixed ? static_cast<int>((budget - fixed) / stream_stage_bytes(mp)) : 0;
+  return st > kStreamMaxStages ? kStreamMaxStages : st;
+}
+
+// Small-batch gate pass (gp.mp, gp.stages set by the caller).
+cudaError_t launch_gate_stream(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GateStreamParams& gp, int* ctrl,
+                               int grid, cudaStream_t s) {
+  const size_t smem = stream_smem_bytes(gp.mp, gp.stages);
+  if (gp.stages < 2 || smem > 232448) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(gate_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(gate_stream_kernel, grid, 192, smem, s, tm_w, tm_x, gp, ctrl);
+}
+
+// Start of a gate pass (both paths): control words, row slots and, for small
+// batches, the tile tickets.
+cudaError_t launch_reset(const twell_buf* tw, cudaStream_t s) {
+  const bool small = tw->z != nullptr;
+  const int n_tickets = small ? tw->N / tw->T : 0;
+  const int rwork = tw->M > n_tickets ? tw->M : n_tickets;
+  const int rgrid = (rwork + 255) / 256 < 1024 ? (rwork + 255) / 256 : 1024;
+  return launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, s, tw->row_slot, tw->M, tw->ctrl,
+                    small ? small_tickets(tw) : nullptr, n_tickets);
+}
+
+GateTwellParams gate_twell_params(const uint16_t* x, const twell_buf* tw) {
+  GateTwellParams p;
+  p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.dense_rows = tw->dense_rows;
+  p.row_slot = tw->row_slot; p.slot_row = tw->slot_row; p.x = x; p.x_over = tw->x_over;
+  p.N = tw->N; p.K = tw->K; p.C = tw->C; p.r_cap = tw->R_cap;
+  return p;
+}
+
+// Tensor maps, parameters and grid of the small-batch gate pass: stream-K over
+// W_g with the tokens on the narrow side of the tile, ranges of at least a
+// third of a tile's k blocks (so at most kStreamSlots CTAs meet a tile), at
+// most one CTA per SM.
+twell_status small_gate_plan(const uint16_t* x, const uint16_t* wg_t, const twell_buf* tw, int sms, size_t smem_budget,
+                             CUtensorMap& tm_w, CUtensorMap& tm_x, GateStreamParams& gp, int& grid) {
+  const int M = tw->M, K = tw->K, N = tw->N;
+  const int mp = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  twell_status st;
+  if ((st = tmap_bf16(wg_t, K, N, 128, tm_w)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(x, K, M, mp, tm_x)) != TWELL_OK) return st;
+  gp.pk = gate_twell_params(x, tw);
+  gp.part = tw->z;
+  gp.tickets = small_tickets(tw);
+  gp.M = M;
+  gp.T = tw->T;
+  gp.kb = K / kBK;
+  gp.units = static_cast<int64_t>(N / 128) * gp.kb;
+  gp.mp = mp;
+  gp.stages = stream_stages(mp, smem_budget);
+  const int64_t pmin = (gp.kb + 2) / 3;
+  const int64_t by_len = gp.units / pmin;
+  grid = static_cast<int>(by_len < sms ? (by_len > 0 ? by_len : 1) : sms);
+  gp.grid = grid;
+  return TWELL_OK;
+}
+
+// Small-batch up/down parameters for `warps_total` warps (each with `stages`
+// ring stages and the full entry list).
+UpdownParams small_updown_params(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
+                                 float* y, int stages, int64_t warps_total) {
+  UpdownParams p = {};
+  p.x = x; p.wu_t = wu_t; p.wd = wd;
+  p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals;
+  p.M = tw->M; p.K = tw->K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
+  p.y = y; p.ctrl = tw->ctrl;
+  p.stages = stages;
+  p.list_cap = kUpdownListCap;
+  p.row_slot = tw->row_slot;
+  p.dense_rows = tw->dense_rows;
+  p.scan_target = 0;
+  p.wait_limit_ns = kWaitLimitNs;
+  // About one unit per warp, each within the list (tiles * C <= list) and one ballot (<= 32 tiles).
+  const int NT = tw->N / tw->T;
+  const int64_t records = static_cast<int64_t>(tw->M) * NT;
+  int tpu = static_cast<int>((records + warps_total - 1) / warps_total);
+  const int tpu_max = kUpdownListCap / tw->C < 32 ? kUpdownListCap / tw->C : 32;
+  p.tiles_per_unit = tpu < 1 ? 1 : (tpu > tpu_max ? tpu_max : tpu);
+  return p;
+}
+
+template <int KV>
+cudaError_t launch_fused_small_kv(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GateStreamParams& gp,
+                                  const UpdownParams& up, int* ctrl, int grid, size_t smem, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(twell_fused_small_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(twell_fused_small_kernel<KV>, grid, 192, smem, s, tm_w, tm_x, gp, up, ctrl);
+}
+
+cudaError_t launch_fused_small(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GateStreamParams& gp,
+                               const UpdownParams& up, int* ctrl, int grid, size_t smem, cudaStream_t s) {
+  switch ((up.K + 255) / 256) {
+#define TW_KV(n) \
+  case n:        \
+    return launch_fused_small_kv<n>(tm_w, tm_x, gp, up, ctrl, grid, smem, s);
+    TW_KV(1) TW_KV(2) TW_KV(3) TW_KV(4) TW_KV(5) TW_KV(6) TW_KV(7) TW_KV(8)
+    TW_KV(9) TW_KV(10) TW_KV(11) TW_KV(12) TW_KV(13) TW_KV(14) TW_KV(15) TW_KV(16)
+#undef TW_KV
+    default:
+      return cudaErrorInvalidValue;
   }
 }
 
@@ -300,7 +349,7 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
   cudaError_t e = cudaFuncSetAttribute(twell_updown_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  UpdownParams p;
+  UpdownParams p = {};
   p.x = x; p.wu_t = wu_t; p.wd = wd;
   p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals;
   p.M = tw->M; p.K = tw->K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
@@ -315,6 +364,44 @@ cudaError_t launch_updown_kv(const uint16_t* x, const uint16_t* wu_t, const uint
     g_expire_wait_ns = 0;
   }
   return launch_pdl(twell_updown_kernel<KV>, sms, 32 * u.warps, smem, s, p);
+}
+
+// Small batches: the static-unit kernel with the full entry list (it must
+// hold one overflow tile, T entries) and two to four ring stages per warp.
+template <int KV>
+cudaError_t launch_updown_small_kv(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
+                                   float* y, int sms, cudaStream_t s) {
+  constexpr size_t kBudget = 232448;
+  const size_t slot = 4 * static_cast<size_t>(tw->K);
+  const size_t fixed = static_cast<size_t>(kUpdownListCap) * 8 + 128;
+  int warps = updown_max_warps<KV>(), stages = 0;
+  for (; warps >= 4; warps = warps > 8 ? 8 : warps / 2) {
+    const size_t per_warp = kBudget / warps;
+    stages = per_warp > fixed ? static_cast<int>((per_warp - fixed) / slot) : 0;
+    if (stages >= 2) break;
+  }
+  if (stages < 2) return cudaErrorInvalidValue;
+  if (stages > 4) stages = 4;
+  const size_t smem = static_cast<size_t>(warps) * updown_warp_bytes(tw->K, stages, kUpdownListCap);
+  cudaError_t e = cudaFuncSetAttribute(twell_updown_small_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const UpdownParams p = small_updown_params(x, wu_t, wd, tw, y, stages, static_cast<int64_t>(sms) * warps);
+  return launch_pdl(twell_updown_small_kernel<KV>, sms, 32 * warps, smem, s, p);
+}
+
+cudaError_t launch_updown_small(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
+                                float* y, int sms, cudaStream_t s) {
+  switch ((tw->K + 255) / 256) {
+#define TW_KV(n) \
+  case n:        \
+    return launch_updown_small_kv<n>(x, wu_t, wd, tw, y, sms, s);
+    TW_KV(1) TW_KV(2) TW_KV(3) TW_KV(4) TW_KV(5) TW_KV(6) TW_KV(7) TW_KV(8)
+    TW_KV(9) TW_KV(10) TW_KV(11) TW_KV(12) TW_KV(13) TW_KV(14) TW_KV(15) TW_KV(16)
+#undef TW_KV
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_updown(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw, float* y,
@@ -472,45 +559,27 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
   DeviceInfo dev;
   if ((st = device_info(dev)) != TWELL_OK) return st;
 
-  // 256-wide CTA tiles halve the operand traffic per FLOP; 128-wide ones give
-  // small-M problems twice the CTAs.
+  const bool small = tw->z != nullptr;
+  // 256-wide CTA tiles halve the operand traffic per FLOP of the one-CTA engine.
   const int bn = (N % 256 == 0 && (M > 256 || tw->T == 256)) ? 256 : 128;
   CUtensorMap tm_x, tm_wg;
-  if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
-  if ((st = tmap_bf16(wg_t, K, N, bn, tm_wg)) != TWELL_OK) return st;
-
-  const bool small = tw->z != nullptr;
-  const int64_t z4 = small ? static_cast<int64_t>(M) * N / 4 : 0;
-  const int64_t rwork = (z4 > M ? z4 : M);
-  const int rgrid = static_cast<int>((rwork + 255) / 256 < 1024 ? (rwork + 255) / 256 : 1024);
+  if (!small) {
+    if ((st = tmap_bf16(x, K, M, kBM, tm_x)) != TWELL_OK) return st;
+    if ((st = tmap_bf16(wg_t, K, N, bn, tm_wg)) != TWELL_OK) return st;
+  }
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_pdl(twell_reset_kernel, rgrid > 0 ? rgrid : 1, 256, 0, stream, tw->row_slot, M, tw->ctrl,
-                     reinterpret_cast<float4*>(tw->z), z4));
+  TW_CUDA(launch_reset(tw, stream));
   TW_CUDA(trace_end(stream, "twell_reset"));
 
-  GateTwellParams p;
-  p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.dense_rows = tw->dense_rows;
-  p.row_slot = tw->row_slot; p.slot_row = tw->slot_row; p.x = x; p.x_over = tw->x_over;
-  p.N = N; p.K = K; p.C = tw->C; p.r_cap = tw->R_cap;
+  const GateTwellParams p = gate_twell_params(x, tw);
   if (small) {
-    // One 128-row tile: cut K so that the tiles cover the SMs, add the slices
-    // into z, then pack.
-    CUtensorMap tm_wg128;
-    if ((st = tmap_bf16(wg_t, K, N, 128, tm_wg128)) != TWELL_OK) return st;
-    const int ks = choose_k_splits(M, N, 128, K, dev.sms);
-    EpiStoreF32::Params pz{tw->z, N, N, 1};
-    GemmGeom gz{M, N, K, nullptr, kGateGroupM, 0, ks};
+    CUtensorMap tm_w128, tm_xs;
+    GateStreamParams gp;
+    int grid = 0;
+    if ((st = small_gate_plan(x, wg_t, tw, dev.sms, 232448, tm_w128, tm_xs, gp, grid)) != TWELL_OK) return st;
     TW_CUDA(trace_begin(stream));
-    TW_CUDA(launch_gate_splitk(tm_x, tm_wg128, gz, pz, tw->ctrl, gemm_grid(M, N, 128, dev.sms, ks), stream));
-    TW_CUDA(trace_end(stream, "gate_splitk_gemm"));
-    const int64_t items = static_cast<int64_t>(M) * (N / tw->T);
-    const int pgrid = static_cast<int>((items + 7) / 8);
-    TW_CUDA(trace_begin(stream));
-    if (tw->T == 128)
-      TW_CUDA(launch_pdl(twell_pack_kernel<128>, pgrid, 256, 0, stream, tw->z, p, M, tw->ctrl));
-    else
-      TW_CUDA(launch_pdl(twell_pack_kernel<256>, pgrid, 256, 0, stream, tw->z, p, M, tw->ctrl));
-    TW_CUDA(trace_end(stream, "twell_pack"));
+    TW_CUDA(launch_gate_stream(tm_w128, tm_xs, gp, tw->ctrl, grid, stream));
+    TW_CUDA(trace_end(stream, "gate_stream_pack"));
   } else if (M > 256 && N % 256 == 0 && dev.sms >= 2) {
     // CTA pairs on 256 x 256 tiles: each CTA moves 2/3 of the operand bytes per FLOP.
     CUtensorMap tm_wg128;
@@ -566,6 +635,15 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
   if ((st = device_info(dev)) != TWELL_OK) return st;
   const int N = tw->N;
 
+  if (tw->z) {
+    // Small batch: y cleared, then one kernel for TwELL and overflow tiles alike.
+    TW_CUDA(trace_begin(stream));
+    TW_CUDA(cudaMemsetAsync(y, 0, static_cast<size_t>(tw->M) * K * sizeof(float), stream));
+    TW_CUDA(launch_updown_small(x, wu_t, wd, tw, y, dev.sms, stream));
+    TW_CUDA(trace_end(stream, "twell_updown_small"));
+    return TWELL_OK;
+  }
+
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_updown(x, wu_t, wd, tw, y, dev.sms, stream));
   TW_CUDA(trace_end(stream, "twell_updown"));
@@ -597,6 +675,68 @@ twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16
   TW_CUDA(launch_overflow_down(tm_ho, tm_wd, g2, p2, tw->ctrl, gemm_grid(tw->R_cap, K, 256, dev.sms, ks2_max),
                                stream));
   TW_CUDA(trace_end(stream, "overflow_down_gemm"));
+  return TWELL_OK;
+}
+
+twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd, int M,
+                             int K, int N, twell_buf* tw, float* y, int* n_over_host, cudaStream_t stream) {
+  g_launches = 0;
+  twell_status st = check_buf(tw);
+  if (st != TWELL_OK) return st;
+  if (M != tw->M || K != tw->K || N != tw->N)
+    return fail(TWELL_ERR_INVALID, "shape (%d,%d,%d) does not match the buffer (%d,%d,%d)", M, K, N, tw->M, tw->K, tw->N);
+  if (!aligned16(x) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y))
+    return fail(TWELL_ERR_INVALID, "x, wg_t, wu_t, wd and y must be non-NULL and 16-byte aligned");
+  DeviceInfo dev;
+  if ((st = device_info(dev)) != TWELL_OK) return st;
+
+  if (!tw->z) {
+    // Larger batches: the gate GEMM with its packing epilogue, then the fused up/down kernel.
+    if ((st = twell_gate_pack(x, wg_t, M, K, N, tw, n_over_host, stream)) != TWELL_OK) return st;
+    const int gate_launches = g_launches;
+    if ((st = twell_ffn_fwd(x, wu_t, wd, tw, K, y, stream)) != TWELL_OK) return st;
+    g_launches += gate_launches;
+    return TWELL_OK;
+  }
+
+  // Small batches: one persistent kernel after the reset.
+  constexpr size_t kBudget = 232448;
+  CUtensorMap tm_w, tm_x;
+  GateStreamParams gp;
+  int grid = 0;
+  if ((st = small_gate_plan(x, wg_t, tw, dev.sms, kBudget, tm_w, tm_x, gp, grid)) != TWELL_OK) return st;
+  constexpr int kWarps = 6;
+  const size_t fixed = 1024 + kStreamCtrlBytes;
+  const size_t list_bytes = static_cast<size_t>(kUpdownListCap) * 8 + 128;
+  int stages = static_cast<int>(((kBudget - fixed) / kWarps - list_bytes) / (4 * static_cast<size_t>(K)));
+  if (stages > 4) stages = 4;
+  if (stages < 2 || gp.stages < 2) return fail(TWELL_ERR_INVALID, "K=%d leaves too little shared memory", K);
+  // Every SM takes part in the up/down phase; the first gp.grid CTAs also in the gate pass.
+  grid = dev.sms;
+  UpdownParams up = small_updown_params(x, wu_t, wd, tw, y, stages, static_cast<int64_t>(grid) * kWarps);
+  up.scan_target = grid;
+  if (g_expire_wait_ns > 0) {
+    up.scan_target = grid + 1;
+    up.wait_limit_ns = static_cast<unsigned long long>(g_expire_wait_ns);
+    g_expire_wait_ns = 0;
+  }
+  const size_t ring = fixed + kWarps * updown_warp_bytes(K, stages, kUpdownListCap);
+  const size_t gate = stream_smem_bytes(gp.mp, gp.stages);
+  const size_t smem = ring > gate ? ring : gate;
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_reset(tw, stream));
+  TW_CUDA(trace_end(stream, "twell_reset"));
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_fused_small(tm_w, tm_x, gp, up, tw->ctrl, grid, smem, stream));
+  TW_CUDA(trace_end(stream, "twell_fused_small"));
+
+  if (n_over_host) {
+    int n_over = 0;
+    if ((st = twell_read_status(tw, &n_over, nullptr, stream)) == TWELL_ERR_DEVICE_CHECK) return st;
+    *n_over_host = n_over;
+    if (n_over > tw->R_cap)
+      return fail(TWELL_ERR_CAPACITY, "%d rows overflowed, dense-row capacity is %d", n_over, tw->R_cap);
+  }
   return TWELL_OK;
 }
 

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         "twell_buf_init": (I, [BP, P, S, I, I, I, I, I, I]),
         "twell_gate_pack": (I, [P, P, I, I, I, BP, IP, P]),
         "twell_ffn_fwd": (I, [P, P, P, BP, I, P, P]),
+        "twell_ffn_fused": (I, [P, P, P, P, I, I, I, BP, P, IP, P]),
         "twell_read_status": (I, [BP, IP, IP, P]),
         "dense_ffn_fwd": (I, [P, P, P, P, I, I, I, P, P, P]),
         "dense_ffn_fwd_bf16h": (I, [P, P, P, P, I, I, I, P, P, P]),
@@ -250,6 +251,29 @@ def ffn_fwd(x: torch.Tensor, wu_t: torch.Tensor, wd: torch.Tensor, tw: TwellBuff
     return y
 
 
+def ffn_fused(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd: torch.Tensor, tw: TwellBuffers,
+              y: Optional[torch.Tensor] = None, sync: bool = False, stream=None) -> torch.Tensor:
+    """twell_ffn_fused: the whole sparse forward in one call (one persistent
+    kernel after the reset for M <= TWELL_SMALL_M).  With sync=True raises
+    CapacityError when the dense-row slots ran out."""
+    M, K = x.shape
+    N = wg_t.shape[0]
+    if y is None:
+        y = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    if y.dtype != torch.float32 or not y.is_contiguous() or tuple(y.shape) != (M, K):
+        raise ValueError("y must be a contiguous float32 tensor of shape (M, K)")
+    L = lib()
+    n_over = ctypes.c_int(-1)
+    st = L.twell_ffn_fused(_bf16(x, "x", (M, K)), _bf16(wg_t, "wg_t", (N, K)), _bf16(wu_t, "wu_t", (N, K)),
+                           _bf16(wd, "wd", (N, K)), M, K, N, ctypes.byref(tw.buf), y.data_ptr(),
+                           ctypes.byref(n_over) if sync else None, _stream(stream))
+    if st == ERR_CAPACITY:
+        raise CapacityError(st, "twell_ffn_fused", (L.twell_last_error() or b"").decode(), n_over.value)
+    _check(st, "twell_ffn_fused")
+    tw.n_over_known = n_over.value if sync else None
+    return y
+
+
 def read_status(tw: TwellBuffers, stream=None):
     """Synchronise and return (status, n_over, device_flags)."""
     n = ctypes.c_int(0)
@@ -298,7 +322,8 @@ def dense_ffn_noalloc(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, w
 
 
 def test_expire_wait(limit_ns: int) -> None:
-    """twell_test_expire_wait: arm a one-shot expiring device wait for the next ffn_fwd."""
+    """twell_test_expire_wait: arm a one-shot expiring device wait for the next
+    ffn_fwd (large batches) or ffn_fused (small batches)."""
     _check(lib().twell_test_expire_wait(int(limit_ns)), "twell_test_expire_wait")
 
 

@@ -13,6 +13,9 @@
  *                     (Tile-wise ELLPACK), never writing the dense gate;
  *   twell_ffn_fwd   : fused up + down projection that visits only the active
  *                     hidden units: y_m = sum_{n in A_m} g_{m,n} (x_m W_u[:,n]) W_d[n,:].
+ * twell_ffn_fused runs both steps in one call; for small batches in one
+ * persistent kernel (the one-pass inference kernel of the summary page
+ * alanhou.org, "Inference Kernels").
  * Tiles whose active count exceeds the capacity C are routed to a dense-row
  * backup (§3-6 hybrid format; §4-3 static capacity of at most M/8 rows,
  * overflow reported to the host, which retries with larger storage).
@@ -71,13 +74,17 @@ typedef enum {
  *   ctrl       int32  [64]        device control words: [0] n_over (rows that
  *                                 asked for a slot), [1] status flags, [2..6]
  *                                 work-queue counters of the fused kernel, [7]
- *                                 entries of the non-overflow tiles
+ *                                 entries of the non-overflow tiles, [8] grid
+ *                                 barrier of twell_ffn_fused's small-batch kernel
  *   x_over     bf16   [R_cap][K]  scratch: gathered x rows of slotted rows
  *   h_over     bf16   [R_cap][2N] scratch: overflow-tile hidden activations as
  *                                 bf16 hi (columns < N) + lo (columns >= N) parts
  *   units      int32  [M*NT][4]   scratch: work units of rows split across warps
- *   z          fp32   [M][N]      scratch, only for M <= TWELL_SMALL_M (else NULL):
- *                                 the gate pre-activation of the small-M path
+ *   z          fp32   [4][M][N] + int32 [NT]
+ *                                 scratch, only for M <= TWELL_SMALL_M (else NULL):
+ *                                 partial gate sums of the small-batch gate pass
+ *                                 (up to four CTAs per 128-unit tile), then one
+ *                                 ticket per TwELL tile
  */
 typedef struct twell_buf {
   uint16_t* counts;
@@ -94,9 +101,12 @@ typedef struct twell_buf {
   int M, K, N, T, C, R_cap;
 } twell_buf;
 
-/* Batches of at most this many rows take the small-M gate path: a split-K
- * gate GEMM into the fp32 scratch z, then a separate TwELL packing kernel
- * (one 128-row tile cannot occupy the GPU otherwise). */
+/* Batches of at most this many rows take the small-batch path.  The gate pass
+ * streams W_g through the tensor cores with the tokens on the narrow side of
+ * the tile (128 hidden units x up to 128 tokens), cut into equal contiguous
+ * k ranges per SM; the last CTA to finish a TwELL tile packs it.  The up/down
+ * pass splits the work statically into (row, tile group) units, one kernel for
+ * TwELL and overflow tiles alike (no dense-row GEMMs). */
 #define TWELL_SMALL_M 128
 
 /* Bytes of device memory twell_buf_init needs for these sizes (0 if invalid). */
@@ -117,9 +127,9 @@ twell_status twell_buf_init(twell_buf* tw, void* base, size_t bytes, int M, int 
  * Transformer Language Models", §3-4 steps 1-5, §3-6, §4-3).  x [M][K], wg_t
  * [N][K] device bf16.  M, K, N must equal the buffer's.  Fills every array of
  * `tw` described above.  Launches: a small reset kernel, then one gate GEMM
- * whose epilogue packs TwELL; for M <= TWELL_SMALL_M instead a split-K gate
- * GEMM into z and a packing kernel (the same records, order and overflow
- * routing).
+ * whose epilogue packs TwELL; for M <= TWELL_SMALL_M instead the small-batch
+ * gate pass described at TWELL_SMALL_M (the same records, order, counts and
+ * overflow routing).
  *
  * n_over_host: if NULL the call is fully asynchronous; the overflow count stays
  * on the device (ctrl[0]) and twell_read_status reports it later.  If not NULL
@@ -136,12 +146,30 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
  * Transformer Language Models", §3-5; filled by twell_gate_pack on the same
  * stream), then the dense-row path for overflow tiles (§3-6, §4-3).  wu_t, wd [N][K]
  * device bf16; y [M][K] device fp32, fully overwritten.  K must equal tw->K.
- * Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
+ * For M <= TWELL_SMALL_M: y is cleared (a memset on `stream`) and one
+ * static-unit kernel serves TwELL and overflow tiles.  Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
  * -2 in row_slot miss their overflow tiles and twell_read_status returns
  * TWELL_ERR_CAPACITY.
  */
 twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
                            int K, float* y, cudaStream_t stream);
+
+/*
+ * The whole sparse forward in one call: x [M][K], wg_t, wu_t, wd [N][K] device
+ * bf16, y [M][K] device fp32 (overwritten); M, K, N must equal the buffer's.
+ * For M <= TWELL_SMALL_M it launches the reset kernel and then one persistent
+ * kernel (one CTA per SM at most, 192 threads) that runs the small-batch gate
+ * pass, waits at a grid barrier (bounded: a wait that gives up raises a device
+ * flag and the CTA returns, so twell_read_status then reports
+ * TWELL_ERR_DEVICE_CHECK), and runs the small-batch up/down units; `tw` holds
+ * the TwELL records afterwards as after twell_gate_pack.  For larger M it is
+ * twell_gate_pack followed by twell_ffn_fwd.  n_over_host as for
+ * twell_gate_pack, except that on small batches the capacity check runs after
+ * the forward (a TWELL_ERR_CAPACITY result leaves y incomplete; retry with a
+ * larger R_cap).
+ */
+twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd, int M,
+                             int K, int N, twell_buf* tw, float* y, int* n_over_host, cudaStream_t stream);
 
 /*
  * Synchronises `stream` and reads the buffer's device control words.
@@ -207,7 +235,10 @@ twell_status dense_ffn_fwd_noalloc(const uint16_t* x, const uint16_t* wg_t, cons
  * with a wait limit of limit_ns nanoseconds instead of the usual 2 s.  The
  * wait expires, the kernel raises its timeout flag and returns (the rows of
  * split work units are then left incomplete), and twell_read_status reports
- * TWELL_ERR_DEVICE_CHECK.  The next twell_gate_pack clears the flag.  No
+ * TWELL_ERR_DEVICE_CHECK.  On a small batch the one-shot is taken instead by
+ * the next twell_ffn_fused, whose grid barrier then waits for one CTA more
+ * than the grid holds (y is left unwritten past the barrier).  The
+ * small-batch twell_ffn_fwd has no such wait and leaves the one-shot armed.  The next twell_gate_pack clears the flag.  No
  * memory access changes.  limit_ns must lie in [1000, 1000000000]; 0 disarms.
  */
 twell_status twell_test_expire_wait(long long limit_ns);

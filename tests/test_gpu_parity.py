@@ -130,13 +130,15 @@ def test_all_gates_off_gives_exact_zero():
     assert torch.count_nonzero(y).item() == 0
 
 
-def test_all_gates_on_routes_every_tile_to_dense_rows():
-    w, d, dev = _small(130, 128, 512, 128, 4, bias=-1e2, seed=2, R_cap=130)
-    t, n_over, y = _run_sparse(dev, w, R_cap=130)
-    assert n_over == 130
+@pytest.mark.parametrize("M", [130, 40])
+def test_all_gates_on_routes_every_tile_to_dense_rows(M):
+    # M = 130: dense-row GEMMs; M = 40: the small-batch kernel serves the slots.
+    w, d, dev = _small(M, 128, 512, 128, 4, bias=-1e2, seed=2, R_cap=M)
+    t, n_over, y = _run_sparse(dev, w, R_cap=M)
+    assert n_over == M
     h = t.to_host()
     assert (h["counts"] == 128).all()
-    _compare(w, d, t, y, np.arange(130))
+    _compare(w, d, t, y, np.arange(M))
 
 
 def test_capacity_equal_tile_never_overflows():
@@ -232,15 +234,29 @@ def test_kernel_trace_brackets_every_launch():
     assert all(ms > 0 for _, ms in tr.times_ms())
 
 
-def test_small_batch_takes_the_split_k_gate_path():
-    # M <= TWELL_SMALL_M: split-K gate GEMM into the fp32 scratch, then the packing kernel.
+def test_small_batch_takes_the_stream_path():
+    # M <= TWELL_SMALL_M: the stream-K gate kernel packs TwELL itself; y is
+    # cleared and one static-unit kernel serves TwELL and overflow tiles.
     w, d, dev = _workload("sweep_m64_k2048_n8192_p99")
     t = tw.TwellBuffers(w.M, w.K, w.N, w.T, w.C)
     with tw.KernelTrace(capacity=8) as tr:
         tw.gate_pack(dev["x"], dev["wg_t"], t)
+        assert tw.last_launch_count() == 2
+        y = tw.ffn_fwd(dev["x"], dev["wu_t"], dev["wd"], t)
+        assert tw.last_launch_count() == 1
     torch.cuda.synchronize()
-    assert [n for n, _ in tr.times_ms()] == ["twell_reset", "gate_splitk_gemm", "twell_pack"]
-    assert tw.last_launch_count() == 3
+    assert [n for n, _ in tr.times_ms()] == ["twell_reset", "gate_stream_pack", "twell_updown_small"]
+    _compare(w, d, t, y, np.arange(w.M))
+
+
+@pytest.mark.parametrize("K,N,T", [(192, 256, 128), (192, 512, 256), (4096, 1024, 256)])
+def test_small_batch_gate_pieces_from_several_ctas(K, N, T):
+    # Few k blocks per 128-unit tile: every tile's sum is split over two to
+    # four CTAs and added by the last one, for T = 128 and for T = 256 (a
+    # TwELL tile spans two 128-unit tiles).
+    w, d, dev = _small(24, K, N, T, 8, None, seed=K + N, R_cap=24)
+    t, n_over, y = _run_sparse(dev, w, R_cap=24)
+    _compare(w, d, t, y, np.arange(24))
 
 
 def test_maximum_sizes_on_both_gate_paths():
