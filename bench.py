@@ -14,7 +14,11 @@ every timed step; the flush is outside the timed events.
 
 The headline workload is the largest single-GPU configuration at 99%
 sparsity (M=16384, K=2560, N=10240); the M=2048 and M=8192 workloads are
-timed the same way and reported under "other_workloads".
+timed the same way and reported under "other_workloads".  Small batches
+(M=16 and M=64 rows, K=2048, N=8192, 99% sparsity) are reported under
+"small_batch": there every step is replayed from a CUDA graph (the launch
+path of a decode loop) and four copies of the weights (4 x 100 MB, more than
+L2) are used in turn, so no step finds its weights in L2.
 
 For N > 1 (torchrun, one rank per GPU) every rank runs its own batch of the
 same workload: the forward pass is token-parallel and needs no collective
@@ -52,6 +56,9 @@ PROFILES = os.path.join(ROOT, "profiles")
 # Timed next to the headline workload and reported under "other_workloads".
 EXTRA_WORKLOADS = ("m2048_k1536_n4096_p99_lognormal05", "m8192_k2048_n5632_loguniform_lognormal07")
 FLUSH_BYTES = 256 << 20
+# Small-batch workloads, timed from CUDA graphs over rotating weight copies.
+SMALL_BATCH_WORKLOADS = ("sweep_m16_k2048_n8192_p99", "sweep_m64_k2048_n8192_p99")
+SMALL_BATCH_COPIES = 4
 
 
 def load_peaks():
@@ -447,6 +454,73 @@ def measure_workload(tw, torch, dev, w, d, steps, warmup, flush, peaks, peak_kin
     return out
 
 
+def measure_small_batch(tw, torch, dev, w, d, peaks, reps=25):
+    """Per-step time of the small-batch paths: twell_ffn_fused (one persistent
+    kernel after the reset), the two-call path (gate_pack + ffn_fwd) and both
+    dense FFNs, each replayed from a CUDA graph of SMALL_BATCH_COPIES steps,
+    step i on weight copy i (their total exceeds L2)."""
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    M, K, N, T, C = w.M, w.K, w.N, w.T, w.C
+    x = to_dev(d["x"])
+    base = [to_dev(d[k]) for k in ("wg_t", "wu_t", "wd")]
+    sets = [base] + [[t.clone() for t in base] for _ in range(SMALL_BATCH_COPIES - 1)]
+    bufs = [tw.TwellBuffers(M, K, N, T, C, device=dev) for _ in range(SMALL_BATCH_COPIES)]
+    ys = [torch.empty(M, K, dtype=torch.float32, device=dev) for _ in range(SMALL_BATCH_COPIES)]
+    h = torch.empty(M, 2 * N, dtype=torch.bfloat16, device=dev)
+    h1 = h.view(-1)[:M * N].view(M, N)
+
+    def fused(i):
+        tw.ffn_fused(x, *sets[i], bufs[i], ys[i])
+
+    def two_call(i):
+        tw.gate_pack(x, sets[i][0], bufs[i])
+        tw.ffn_fwd(x, sets[i][1], sets[i][2], bufs[i], ys[i])
+
+    def dense(i):
+        tw.dense_ffn(x, *sets[i], h, ys[i])
+
+    def dense1(i):
+        tw.dense_ffn(x, *sets[i], h1, ys[i], bf16_h=True)
+
+    out = {"workload": w.name, "M": M, "K": K, "N": N, "T": T, "C": C,
+           "timing": f"CUDA graph of {SMALL_BATCH_COPIES} steps on {SMALL_BATCH_COPIES} weight copies "
+                     f"({SMALL_BATCH_COPIES * 6 * K * N / 1e6:.0f} MB, more than L2), {reps} replays"}
+    for name, fn in (("fused", fused), ("two_call", two_call), ("dense", dense), ("dense_bf16h", dense1)):
+        for i in range(SMALL_BATCH_COPIES):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(SMALL_BATCH_COPIES):
+                fn(i)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        b.synchronize()
+        out[name] = {"ms_per_step": a.elapsed_time(b) / (reps * SMALL_BATCH_COPIES)}
+        del g
+    st, n_over, flags = tw.read_status(bufs[0])
+    if st != tw.OK:
+        raise RuntimeError(f"{w.name}: small-batch status {st} flags {flags}")
+    U = unique_active_units(bufs[0], C, T)
+    ms = out["fused"]["ms_per_step"]
+    out["value"] = M / (ms * 1e-3)
+    out["unit"] = UNIT
+    out["n_over"] = n_over
+    out["unique_units_gathered"] = U
+    out["path_roofline"] = path_roofline(M, K, N, T, C, U, n_over, peaks, ms)
+    out["speedup_vs_dense"] = out["dense"]["ms_per_step"] / ms
+    out["speedup_vs_dense_bf16h"] = out["dense_bf16h"]["ms_per_step"] / ms
+    return out
+
+
 def run_ncu_case(args):
     """The sparse path only, --warmup + 1 times, on one GPU: the launches an
     ncu capture selects from (no flush buffer, no dense FFN, no timing)."""
@@ -528,6 +602,13 @@ def run_native(args, rank, world, local_rank):
             others[name] = r
             torch.cuda.empty_cache()
 
+    small = {}
+    if not args.no_extra:
+        for name in SMALL_BATCH_WORKLOADS:
+            ws = wl.WORKLOADS[name]
+            small[name] = measure_small_batch(tw, torch, dev, ws, wl.generate(ws), peaks)
+            torch.cuda.empty_cache()
+
     # One collective on every rank: the job's time is the slowest rank's.
     ms, e2e_ms = max_over_ranks([head["ms_per_step"], e2e_ms], world, dev)
     if rank != 0:
@@ -565,6 +646,7 @@ def run_native(args, rank, world, local_rank):
         "gpu_launches": head["gpu_launches"],
         "clocks": clk.summary(),
         "other_workloads": others,
+        "small_batch": small,
     }
     print(json.dumps(line), flush=True)
 
