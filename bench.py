@@ -534,12 +534,16 @@ def run_ncu_case(args):
     tb = tw.TwellBuffers(w.M, w.K, w.N, w.T, w.C)
     y = torch.empty(w.M, w.K, dtype=torch.float32, device="cuda")
     for _ in range(args.warmup + 1):
-        tw.gate_pack(dev["x"], dev["wg_t"], tb)
-        tw.ffn_fwd(dev["x"], dev["wu_t"], dev["wd"], tb, y)
+        if args.ncu_fused:
+            tw.ffn_fused(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"], tb, y)
+        else:
+            tw.gate_pack(dev["x"], dev["wg_t"], tb)
+            tw.ffn_fwd(dev["x"], dev["wu_t"], dev["wd"], tb, y)
     st, n_over, flags = tw.read_status(tb)
     if st != tw.OK:
         raise RuntimeError(f"status {st} (n_over {n_over}, flags {flags})")
-    print(json.dumps({"ncu_case": w.name, "passes": args.warmup + 1, "n_over": n_over}))
+    print(json.dumps({"ncu_case": w.name, "passes": args.warmup + 1, "n_over": n_over,
+                      "call": "twell_ffn_fused" if args.ncu_fused else "twell_gate_pack + twell_ffn_fwd"}))
 
 
 def run_native(args, rank, world, local_rank):
@@ -662,6 +666,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="time only --workload")
     ap.add_argument("--ncu-case", action="store_true",
                     help="no timing: --warmup + 1 passes of the sparse path on --workload (for ncu captures)")
+    ap.add_argument("--ncu-fused", action="store_true", help="with --ncu-case: the passes call twell_ffn_fused")
     args = ap.parse_args()
     if args.warmup < 3 and not args.ncu_case:
         ap.error("--warmup must be >= 3")
