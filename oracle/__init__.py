@@ -10,7 +10,9 @@ Every function takes bf16 bit patterns (``uint16`` numpy arrays, layouts as in
 ``activation_sparse_gated_tma_b200.workloads``) and returns float64 results.
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (library-routine cross-checks, closed forms, invariants and a hand-worked
-golden example); none is "parity unpinned".
+golden example); none is "parity unpinned".  The backward pass lives in
+``oracle.backward`` (numpy float64), pinned there by central differences of
+the float64 forward.
 """
 from __future__ import annotations
 

@@ -247,3 +247,63 @@ def test_generator_truncation_keeps_prefix():
     part = wl.generate(wl.TINY_WORKLOAD, M=10)
     assert np.array_equal(full["x"][:10], part["x"])
     assert np.array_equal(full["wg_t"], part["wg_t"])
+
+
+# ---------------------------------------------------------------- backward oracle
+from oracle import backward as ob  # noqa: E402
+
+
+def _fd_problem(seed):
+    """A tiny float64 problem whose gate pre-activations all stay at least 0.05
+    away from 0, so that central differences never cross a ReLU kink."""
+    for s in range(seed, seed + 500):
+        rng = np.random.default_rng(s)
+        M, K, N = 3, 8, 6
+        X = rng.standard_normal((M, K))
+        G = rng.standard_normal((N, K)) / np.sqrt(K)
+        U = rng.standard_normal((N, K)) / np.sqrt(K)
+        D = rng.standard_normal((N, K)) / np.sqrt(N)
+        z = X @ G.T
+        if np.abs(z).min() > 0.05 and 0 < (z > 0).sum() < z.size:
+            return X, G, U, D, rng.standard_normal((M, K))
+    raise AssertionError("no problem without kinks found")
+
+
+@pytest.mark.parametrize("seed", [0, 100, 200])
+def test_backward_matches_central_differences_of_the_forward(seed):
+    # L = sum(R * y): dL/dy = R.  Every entry of x and of the three weights is
+    # perturbed by +-eps in the plain float64 forward.
+    X, G, U, D, R = _fd_problem(seed)
+    got = ob.backward_f64(X, G, U, D, R)
+    eps = 1e-6
+    for name, A, key in (("x", X, "dx"), ("wg_t", G, "dwg_t"), ("wu_t", U, "dwu_t"), ("wd", D, "dwd")):
+        fd = np.empty_like(A)
+        for i in np.ndindex(A.shape):
+            keep = A[i]
+            A[i] = keep + eps
+            lp = np.sum(R * ob.ffn_forward_f64(X, G, U, D))
+            A[i] = keep - eps
+            lm = np.sum(R * ob.ffn_forward_f64(X, G, U, D))
+            A[i] = keep
+            fd[i] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(got[key], fd, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_backward_all_gates_off_is_zero_and_the_mask_argument_is_the_active_set():
+    X, G, U, D, R = _fd_problem(300)
+    off = ob.backward_f64(X, G, U, D, R, active=np.zeros((3, 6), bool))
+    for k in ("dx", "dwg_t", "dwu_t", "dwd"):
+        assert not off[k].any()
+    a = ob.backward_f64(X, G, U, D, R)
+    b = ob.backward_f64(X, G, U, D, R, active=(X @ G.T) > 0)
+    for k in ("dx", "dwg_t", "dwu_t", "dwd"):
+        assert np.array_equal(a[k], b[k])
+
+
+def test_backward_bits_entry_point_widens_bf16_exactly():
+    x, wg, wu, wd, *_ = _rand_problem(4, 64, 128, seed=5)
+    dy = np.random.default_rng(6).standard_normal((4, 64))
+    a = ob.ffn_backward(x, wg, wu, wd, dy)
+    b = ob.backward_f64(_f64(x), _f64(wg), _f64(wu), _f64(wd), dy)
+    for k in ("dx", "dwg_t", "dwu_t", "dwd"):
+        assert np.array_equal(a[k], b[k])
