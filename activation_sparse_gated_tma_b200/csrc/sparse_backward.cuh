@@ -1,0 +1,378 @@
+// Backward pass of the sparse gated FFN over its hybrid activations
+// ("Sparser, Faster, Lighter Transformer Language Models", §3-6 and §3-7:
+// training keeps the activations in the hybrid TwELL + dense-row form, and
+// every backward product visits only the active units).
+//
+// Per token row x with upstream gradient dy, and every active unit n of the
+// row (g = ReLU(z) > 0, taken from TwELL or, for overflow tiles, from the
+// row's dense-row slot):
+//
+//   u = x . W_u^T[n],  dh = dy . W_d[n],  h = u g,  du = dh g,  dz = dh u
+//   dx += du W_u^T[n] + dz W_g^T[n]
+//   dW_d[n] += h dy,  dW_u^T[n] += du x,  dW_g^T[n] += dz x
+//
+// Three passes:
+//   1. count   : active entries per hidden unit (atomic counts);
+//   2. scan    : exclusive prefix of the counts (one CTA) -> each unit's
+//                segment of a unit-major entry list (the hybrid transpose);
+//   3. rows    : static (row, tile group) units as in the small-batch
+//                up/down kernel; the W_u^T, W_d and W_g^T rows of every entry
+//                stream through a per-warp ring; the warp adds du W_u^T + dz
+//                W_g^T into dx (vector atomics, dx cleared first) and appends
+//                (row, h, du, dz) to the unit's segment;
+//   4. units   : one warp per (unit, 256-column chunk) reads the unit's
+//                segment and the entries' x and dy chunks, and writes the
+//                chunk of the three weight-gradient rows (plain stores; units
+//                with no entry get zero rows).
+#pragma once
+
+#include "sparse_updown.cuh"
+
+namespace twell {
+
+struct BwdEntry {
+  int m;
+  float h, du, dz;
+};
+
+struct BwdParams {
+  const uint16_t* x;
+  const uint16_t* wg_t;
+  const uint16_t* wu_t;
+  const uint16_t* wd;
+  const float* dy;
+  const uint16_t* counts;
+  const uint8_t* idx;
+  const float* vals;
+  const int* row_slot;
+  const float* dense_rows;
+  int M, K, N, T, C;
+  float* dx;
+  float* dwg_t;
+  float* dwu_t;
+  float* dwd;
+  int* cnt;            // [N] entries per unit
+  int* off;            // [N + 1] start of each unit's segment
+  int* fill;           // [N] entries written so far per unit
+  BwdEntry* entries;   // unit-major entry list
+  int stages, list_cap, tiles_per_unit;
+  int* ctrl;
+};
+
+// ---------------------------------------------------------------- 1. count
+__global__ void __launch_bounds__(256) twell_bwd_count_kernel(const BwdParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int NT = p.N / p.T;
+  const int64_t records = static_cast<int64_t>(p.M) * NT;
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < records;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c = p.counts[r];
+    if (c == 0) continue;
+    const int m = static_cast<int>(r / NT);
+    const int t = static_cast<int>(r - static_cast<int64_t>(m) * NT);
+    if (c <= p.C) {
+      for (int s = 0; s < c; ++s) atomicAdd(p.cnt + t * p.T + p.idx[r * p.C + s], 1);
+    } else {
+      const int slot = p.row_slot[m];
+      if (slot < 0) continue;
+      const float* g = p.dense_rows + static_cast<int64_t>(slot) * p.N + static_cast<int64_t>(t) * p.T;
+      for (int j = 0; j < p.T; ++j)
+        if (g[j] > 0.f) atomicAdd(p.cnt + t * p.T + j, 1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- 2. scan
+// One CTA of 1024 threads: thread i sums its run of consecutive counts, the
+// CTA scans the 1024 sums, and each thread writes its run's offsets.
+__global__ void __launch_bounds__(1024) twell_bwd_scan_kernel(const BwdParams p) {
+  __shared__ int part[1024];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int per = (p.N + 1023) / 1024;
+  const int a = threadIdx.x * per;
+  const int b = a + per < p.N ? a + per : p.N;
+  int s = 0;
+  for (int n = a; n < b; ++n) s += p.cnt[n];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int v = threadIdx.x >= o ? part[threadIdx.x - o] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int run = part[threadIdx.x] - s;  // exclusive start of this thread's run
+  for (int n = a; n < b; ++n) {
+    p.off[n] = run;
+    run += p.cnt[n];
+  }
+  if (threadIdx.x == 1023) p.off[p.N] = part[1023];
+}
+
+// ---------------------------------------------------------------- 3. rows
+// acc += the products of 8 fp32 values of a and the 8 bf16 values of b.
+__device__ __forceinline__ void dot8_f32_bf16(const float (&a)[8], const uint4& b, float& s0, float& s1) {
+  const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    s0 = fmaf(a[2 * e], __uint_as_float(bw[e] << 16), s0);
+    s1 = fmaf(a[2 * e + 1], __uint_as_float(bw[e] & 0xFFFF0000u), s1);
+  }
+}
+
+// Bytes of one warp's shared memory in the row pass: [ring: stages x (W_u^T row
+// | W_d row | W_g^T row)][list n: int x cap][list g: float x cap].
+__host__ __device__ constexpr size_t bwd_warp_bytes(int K, int stages, int list_cap) {
+  return ((static_cast<size_t>(stages) * 6 * K + static_cast<size_t>(list_cap) * 8) + 127) / 128 * 128;
+}
+
+// Most warps per CTA of the row pass: eight while a lane's x, dy and dx
+// pieces fit the registers of eight warps, else six.
+template <int KV>
+constexpr int bwd_max_warps() {
+  return KV <= 8 ? 8 : 6;
+}
+
+template <int KV>
+__device__ __forceinline__ void bwd_issue(const BwdParams& p, const WarpRing& w, int slot, int n, int lane) {
+  uint4* dst = reinterpret_cast<uint4*>(w.ring + static_cast<size_t>(slot) * w.slot_bytes);
+  const int kv = p.K / 8;
+  const uint4* su = reinterpret_cast<const uint4*>(p.wu_t + static_cast<int64_t>(n) * p.K);
+  const uint4* sd = reinterpret_cast<const uint4*>(p.wd + static_cast<int64_t>(n) * p.K);
+  const uint4* sg = reinterpret_cast<const uint4*>(p.wg_t + static_cast<int64_t>(n) * p.K);
+#pragma unroll
+  for (int j = 0; j < KV; ++j) {
+    const int v = j * 32 + lane;
+    if (v < kv) {
+      cp_async16(dst + v, su + v, w.policy);
+      cp_async16(dst + kv + v, sd + v, w.policy);
+      cp_async16(dst + 2 * kv + v, sg + v, w.policy);
+    }
+  }
+}
+
+// The E listed entries of row m through the ring (one copy group per slot and
+// lane, refilled `stages` entries ahead).
+template <int KV>
+__device__ __forceinline__ void bwd_stream(const BwdParams& p, const WarpRing& w, int E, int m, const uint4 (&xv)[KV],
+                                           const float (&dyv)[KV][8], float (&acc)[KV][8], int lane) {
+  const int S = w.stages;
+  for (int e = 0; e < S; ++e) {
+    if (e < E) bwd_issue<KV>(p, w, e, w.list_n[e], lane);
+    cp_async_commit();
+  }
+  const int kv = p.K / 8;
+  int slot = 0;
+  for (int e = 0; e < E; ++e) {
+    cp_async_wait_pending(S - 1);
+    const uint4* ru = reinterpret_cast<const uint4*>(w.ring + static_cast<size_t>(slot) * w.slot_bytes);
+    const uint4* rd = ru + kv;
+    const uint4* rg = ru + 2 * kv;
+    float qu[4] = {0.f, 0.f, 0.f, 0.f};
+    float qd0 = 0.f, qd1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < KV; ++j) {
+      if (j * 32 + lane < kv) {
+        dot8_acc4(xv[j], ru[j * 32 + lane], qu);
+        dot8_f32_bf16(dyv[j], rd[j * 32 + lane], qd0, qd1);
+      }
+    }
+    float u = (qu[0] + qu[1]) + (qu[2] + qu[3]);
+    float dh = qd0 + qd1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      u += __shfl_xor_sync(0xffffffffu, u, o);
+      dh += __shfl_xor_sync(0xffffffffu, dh, o);
+    }
+    const int n = w.list_n[e];
+    const float g = w.list_g[e];
+    const float du = dh * g;
+    const float dz = dh * u;
+#pragma unroll
+    for (int j = 0; j < KV; ++j) {
+      if (j * 32 + lane < kv) {
+        axpy8_bf16(acc[j], du, ru[j * 32 + lane]);
+        axpy8_bf16(acc[j], dz, rg[j * 32 + lane]);
+      }
+    }
+    if (lane == 0) {
+      const int pos = p.off[n] + atomicAdd(p.fill + n, 1);
+      BwdEntry en;
+      en.m = m;
+      en.h = u * g;
+      en.du = du;
+      en.dz = dz;
+      p.entries[pos] = en;
+    }
+    // This lane has read the slot: refill it with the entry S places ahead.
+    if (e + S < E) bwd_issue<KV>(p, w, slot, w.list_n[e + S], lane);
+    cp_async_commit();
+    slot = slot + 1 == S ? 0 : slot + 1;
+  }
+}
+
+template <int KV>
+__global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_kernel(const BwdParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int NT = p.N / p.T;
+  WarpRing w;
+  w.slot_bytes = 6u * p.K;
+  w.stages = p.stages;
+  w.ring = smem + static_cast<size_t>(warp) * bwd_warp_bytes(p.K, p.stages, p.list_cap);
+  w.list_n = reinterpret_cast<int*>(w.ring + static_cast<size_t>(p.stages) * w.slot_bytes);
+  w.list_g = reinterpret_cast<float*>(w.list_n + p.list_cap);
+  w.list_cap = p.list_cap;
+  w.policy = l2_evict_last_policy();
+  griddep_launch_dependents();
+  griddep_wait();
+
+  // list_entries reads TwELL through the up/down kernel's parameter block.
+  UpdownParams lp = {};
+  lp.counts = p.counts;
+  lp.idx = p.idx;
+  lp.vals = p.vals;
+  lp.N = p.N;
+  lp.T = p.T;
+  lp.C = p.C;
+
+  const int tpu = p.tiles_per_unit;
+  const int groups = (NT + tpu - 1) / tpu;
+  const int64_t n_units = static_cast<int64_t>(p.M) * groups;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  uint4 xv[KV];
+  float dyv[KV][8];
+  float acc[KV][8];
+  for (int64_t u = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; u < n_units; u += stride) {
+    const int row = static_cast<int>(u / groups);
+    const int t0 = static_cast<int>(u - static_cast<int64_t>(row) * groups) * tpu;
+    const int t1 = t0 + tpu < NT ? t0 + tpu : NT;
+    const int c = t0 + lane < t1 ? static_cast<int>(p.counts[static_cast<int64_t>(row) * NT + t0 + lane]) : 0;
+    if (__ballot_sync(0xffffffffu, c > 0) == 0) continue;
+    const uint32_t ov = __ballot_sync(0xffffffffu, c > p.C);
+    const uint16_t* xr = p.x + static_cast<int64_t>(row) * p.K;
+    const float* dyr = p.dy + static_cast<int64_t>(row) * p.K;
+#pragma unroll
+    for (int j = 0; j < KV; ++j) {
+      const int k0 = (j * 32 + lane) * 8;
+      const bool in = k0 < p.K;
+      xv[j] = in ? *reinterpret_cast<const uint4*>(xr + k0) : make_uint4(0, 0, 0, 0);
+      const float4 a = in ? *reinterpret_cast<const float4*>(dyr + k0) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 b = in ? *reinterpret_cast<const float4*>(dyr + k0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      dyv[j][0] = a.x; dyv[j][1] = a.y; dyv[j][2] = a.z; dyv[j][3] = a.w;
+      dyv[j][4] = b.x; dyv[j][5] = b.y; dyv[j][6] = b.z; dyv[j][7] = b.w;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+    }
+    int cursor = t0;
+    while (cursor < t1) {
+      const int E = list_entries(lp, w, row, cursor, t1, lane);
+      if (E > 0) bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
+    }
+    const int slot = ov ? p.row_slot[row] : -1;
+    if (slot >= 0) {
+      uint32_t rest = ov;
+      int E = 0;
+      __syncwarp();
+      while (rest) {
+        const int t = t0 + __ffs(rest) - 1;
+        rest &= rest - 1;
+        if (E + p.T > w.list_cap) {
+          __syncwarp();
+          bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
+          E = 0;
+          __syncwarp();
+        }
+        const float* src = p.dense_rows + static_cast<int64_t>(slot) * p.N + static_cast<int64_t>(t) * p.T;
+        for (int j0 = 0; j0 < p.T; j0 += 32) {
+          const float gv = src[j0 + lane];
+          const uint32_t bal = __ballot_sync(0xffffffffu, gv > 0.f);
+          if (gv > 0.f) {
+            const int pos = E + __popc(bal & ((1u << lane) - 1u));
+            w.list_n[pos] = t * p.T + j0 + lane;
+            w.list_g[pos] = gv;
+          }
+          E += __popc(bal);
+        }
+      }
+      __syncwarp();
+      if (E > 0) bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
+    }
+    float* dxr = p.dx + static_cast<int64_t>(row) * p.K;
+#pragma unroll
+    for (int j = 0; j < KV; ++j) {
+      const int k0 = (j * 32 + lane) * 8;
+      if (k0 < p.K) {
+        atomicAdd(reinterpret_cast<float4*>(dxr + k0), make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]));
+        atomicAdd(reinterpret_cast<float4*>(dxr + k0 + 4), make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]));
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- 4. units
+// Warp item = (unit n, chunk c of 256 columns); lane l holds columns
+// c*256 + 8l .. +8 of the three gradient rows.
+__global__ void __launch_bounds__(256) twell_bwd_units_kernel(const BwdParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int chunks = (p.K + 255) / 256;
+  const int64_t items = static_cast<int64_t>(p.N) * chunks;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+       it += stride) {
+    const int n = static_cast<int>(it / chunks);
+    const int k0 = static_cast<int>(it - static_cast<int64_t>(n) * chunks) * 256 + lane * 8;
+    const bool in = k0 < p.K;
+    float ad[8], au[8], ag[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ad[e] = au[e] = ag[e] = 0.f;
+    const int e0 = p.off[n];
+    const int e1 = p.off[n + 1];
+    for (int b = e0; b < e1; b += 32) {
+      // Lane j holds entry b + j; the warp then walks them in order.
+      BwdEntry mine = {0, 0.f, 0.f, 0.f};
+      if (b + lane < e1) mine = p.entries[b + lane];
+      const int cntb = e1 - b < 32 ? e1 - b : 32;
+      for (int j = 0; j < cntb; ++j) {
+        const int m = __shfl_sync(0xffffffffu, mine.m, j);
+        const float h = __shfl_sync(0xffffffffu, mine.h, j);
+        const float du = __shfl_sync(0xffffffffu, mine.du, j);
+        const float dz = __shfl_sync(0xffffffffu, mine.dz, j);
+        if (in) {
+          const uint4 xq = *reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.K + k0);
+          const float4 d0 = *reinterpret_cast<const float4*>(p.dy + static_cast<int64_t>(m) * p.K + k0);
+          const float4 d1 = *reinterpret_cast<const float4*>(p.dy + static_cast<int64_t>(m) * p.K + k0 + 4);
+          const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+          const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float xlo = __uint_as_float(xw[e] << 16);
+            const float xhi = __uint_as_float(xw[e] & 0xFFFF0000u);
+            au[2 * e] = fmaf(du, xlo, au[2 * e]);
+            au[2 * e + 1] = fmaf(du, xhi, au[2 * e + 1]);
+            ag[2 * e] = fmaf(dz, xlo, ag[2 * e]);
+            ag[2 * e + 1] = fmaf(dz, xhi, ag[2 * e + 1]);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ad[e] = fmaf(h, dv[e], ad[e]);
+        }
+      }
+    }
+    if (in) {
+      const int64_t o = static_cast<int64_t>(n) * p.K + k0;
+      reinterpret_cast<float4*>(p.dwd + o)[0] = make_float4(ad[0], ad[1], ad[2], ad[3]);
+      reinterpret_cast<float4*>(p.dwd + o)[1] = make_float4(ad[4], ad[5], ad[6], ad[7]);
+      reinterpret_cast<float4*>(p.dwu_t + o)[0] = make_float4(au[0], au[1], au[2], au[3]);
+      reinterpret_cast<float4*>(p.dwu_t + o)[1] = make_float4(au[4], au[5], au[6], au[7]);
+      reinterpret_cast<float4*>(p.dwg_t + o)[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
+      reinterpret_cast<float4*>(p.dwg_t + o)[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+    }
+  }
+}
+
+}  // namespace twell

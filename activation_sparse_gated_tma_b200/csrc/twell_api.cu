@@ -13,6 +13,7 @@
 #include "../../include/twell.h"
 #include "internal.h"
 #include "fused_small.cuh"
+#include "sparse_backward.cuh"
 
 namespace twell {
 namespace {
@@ -301,6 +302,66 @@ cudaError_t launch_fused_small(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
     return launch_fused_small_kv<n>(tm_w, tm_x, gp, up, ctrl, grid, smem, s);
     TW_KV(1) TW_KV(2) TW_KV(3) TW_KV(4) TW_KV(5) TW_KV(6) TW_KV(7) TW_KV(8)
     TW_KV(9) TW_KV(10) TW_KV(11) TW_KV(12) TW_KV(13) TW_KV(14) TW_KV(15) TW_KV(16)
+#undef TW_KV
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------- backward
+constexpr int kBwdMaxK = 2560;  // the row pass keeps x, dy and dx pieces of a row in registers
+
+struct BwdLayout {
+  size_t cnt, fill, off, entries, total;
+  int64_t cap;
+};
+
+BwdLayout bwd_layout(int M, int N, int T, int C, int R_cap) {
+  BwdLayout L;
+  L.cap = static_cast<int64_t>(M) * (N / T) * C + static_cast<int64_t>(R_cap) * N;
+  size_t o = 0;
+  L.cnt = o; o = align256(o + size_t(N) * 4);
+  L.fill = o; o = align256(o + size_t(N) * 4);
+  L.off = o; o = align256(o + size_t(N + 1) * 4);
+  L.entries = o; o = align256(o + size_t(L.cap) * sizeof(BwdEntry));
+  L.total = o;
+  return L;
+}
+
+template <int KV>
+cudaError_t launch_bwd_rows_kv(BwdParams p, int sms, cudaStream_t s) {
+  constexpr size_t kBudget = 232448;
+  const size_t list = static_cast<size_t>(kUpdownListCap) * 8 + 128;
+  int warps = bwd_max_warps<KV>(), stages = 0;
+  for (; warps >= 2; --warps) {
+    const size_t per_warp = kBudget / warps;
+    stages = per_warp > list ? static_cast<int>((per_warp - list) / (6 * static_cast<size_t>(p.K))) : 0;
+    if (stages >= 2) break;
+  }
+  if (stages < 2) return cudaErrorInvalidValue;
+  if (stages > 4) stages = 4;
+  p.stages = stages;
+  p.list_cap = kUpdownListCap;
+  // About two units per warp, each within the list and one ballot (<= 32 tiles).
+  const int NT = p.N / p.T;
+  const int64_t records = static_cast<int64_t>(p.M) * NT;
+  const int64_t nw = static_cast<int64_t>(sms) * warps;
+  int tpu = static_cast<int>((records + 2 * nw - 1) / (2 * nw));
+  const int tpu_max = kUpdownListCap / p.C < 32 ? kUpdownListCap / p.C : 32;
+  p.tiles_per_unit = tpu < 1 ? 1 : (tpu > tpu_max ? tpu_max : tpu);
+  const size_t smem = static_cast<size_t>(warps) * bwd_warp_bytes(p.K, stages, kUpdownListCap);
+  cudaError_t e = cudaFuncSetAttribute(twell_bwd_rows_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(twell_bwd_rows_kernel<KV>, sms, 32 * warps, smem, s, p);
+}
+
+cudaError_t launch_bwd_rows(const BwdParams& p, int sms, cudaStream_t s) {
+  switch ((p.K + 255) / 256) {
+#define TW_KV(n) \
+  case n:        \
+    return launch_bwd_rows_kv<n>(p, sms, s);
+    TW_KV(1) TW_KV(2) TW_KV(3) TW_KV(4) TW_KV(5) TW_KV(6) TW_KV(7) TW_KV(8) TW_KV(9) TW_KV(10)
 #undef TW_KV
     default:
       return cudaErrorInvalidValue;
@@ -737,6 +798,64 @@ twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint
     if (n_over > tw->R_cap)
       return fail(TWELL_ERR_CAPACITY, "%d rows overflowed, dense-row capacity is %d", n_over, tw->R_cap);
   }
+  return TWELL_OK;
+}
+
+size_t twell_bwd_scratch_bytes(int M, int K, int N, int T, int C, int R_cap) {
+  if (!shape_ok(M, K, N, T, C, R_cap)) return 0;
+  return bwd_layout(M, N, T, C, R_cap).total;
+}
+
+twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
+                           const twell_buf* tw, const float* dy, int K, float* dx, float* dwg_t, float* dwu_t,
+                           float* dwd, void* scratch, size_t scratch_bytes, cudaStream_t stream) {
+  g_launches = 0;
+  twell_status st = check_buf(tw);
+  if (st != TWELL_OK) return st;
+  if (K != tw->K) return fail(TWELL_ERR_INVALID, "K=%d does not match the buffer's K=%d", K, tw->K);
+  if (K > kBwdMaxK) return fail(TWELL_ERR_INVALID, "twell_ffn_bwd supports K <= %d (got %d)", kBwdMaxK, K);
+  if (!aligned16(x) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(dy) || !aligned16(dx) ||
+      !aligned16(dwg_t) || !aligned16(dwu_t) || !aligned16(dwd))
+    return fail(TWELL_ERR_INVALID, "every array must be non-NULL and 16-byte aligned");
+  const BwdLayout L = bwd_layout(tw->M, tw->N, tw->T, tw->C, tw->R_cap);
+  if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u))
+    return fail(TWELL_ERR_INVALID, "scratch must be non-NULL and 256-byte aligned");
+  if (scratch_bytes < L.total) return fail(TWELL_ERR_INVALID, "scratch too small: %zu < %zu bytes", scratch_bytes, L.total);
+  DeviceInfo dev;
+  if ((st = device_info(dev)) != TWELL_OK) return st;
+
+  uint8_t* sb = static_cast<uint8_t*>(scratch);
+  BwdParams p = {};
+  p.x = x; p.wg_t = wg_t; p.wu_t = wu_t; p.wd = wd; p.dy = dy;
+  p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.row_slot = tw->row_slot; p.dense_rows = tw->dense_rows;
+  p.M = tw->M; p.K = K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
+  p.dx = dx; p.dwg_t = dwg_t; p.dwu_t = dwu_t; p.dwd = dwd;
+  p.cnt = reinterpret_cast<int*>(sb + L.cnt);
+  p.fill = reinterpret_cast<int*>(sb + L.fill);
+  p.off = reinterpret_cast<int*>(sb + L.off);
+  p.entries = reinterpret_cast<BwdEntry*>(sb + L.entries);
+  p.ctrl = tw->ctrl;
+
+  TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // counts and fill
+  TW_CUDA(cudaMemsetAsync(dx, 0, static_cast<size_t>(tw->M) * K * sizeof(float), stream));
+  const int64_t records = static_cast<int64_t>(tw->M) * (tw->N / tw->T);
+  const int64_t cgrid = (records + 255) / 256;
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_pdl(twell_bwd_count_kernel, static_cast<int>(cgrid < 4 * dev.sms ? cgrid : 4 * dev.sms), 256, 0,
+                     stream, p));
+  TW_CUDA(trace_end(stream, "bwd_count"));
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, p));
+  TW_CUDA(trace_end(stream, "bwd_scan"));
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_bwd_rows(p, dev.sms, stream));
+  TW_CUDA(trace_end(stream, "bwd_rows"));
+  const int64_t items = static_cast<int64_t>(tw->N) * ((K + 255) / 256);
+  const int64_t ugrid = (items + 7) / 8;
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_pdl(twell_bwd_units_kernel, static_cast<int>(ugrid < 8 * dev.sms ? ugrid : 8 * dev.sms), 256, 0,
+                     stream, p));
+  TW_CUDA(trace_end(stream, "bwd_units"));
   return TWELL_OK;
 }
 

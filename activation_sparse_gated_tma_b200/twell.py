@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         "twell_gate_pack": (I, [P, P, I, I, I, BP, IP, P]),
         "twell_ffn_fwd": (I, [P, P, P, BP, I, P, P]),
         "twell_ffn_fused": (I, [P, P, P, P, I, I, I, BP, P, IP, P]),
+        "twell_bwd_scratch_bytes": (S, [I, I, I, I, I, I]),
+        "twell_ffn_bwd": (I, [P, P, P, P, BP, P, I, P, P, P, P, P, S, P]),
         "twell_read_status": (I, [BP, IP, IP, P]),
         "dense_ffn_fwd": (I, [P, P, P, P, I, I, I, P, P, P]),
         "dense_ffn_fwd_bf16h": (I, [P, P, P, P, I, I, I, P, P, P]),
@@ -272,6 +274,30 @@ def ffn_fused(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd: torch
     _check(st, "twell_ffn_fused")
     tw.n_over_known = n_over.value if sync else None
     return y
+
+
+def ffn_bwd(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd: torch.Tensor, tw: TwellBuffers,
+            dy: torch.Tensor, scratch: Optional[torch.Tensor] = None, stream=None):
+    """twell_ffn_bwd: (dx, dwg_t, dwu_t, dwd), all fp32, from the forward's TwELL
+    buffer `tw` and the upstream gradient dy [M][K] fp32."""
+    M, K = x.shape
+    N = wg_t.shape[0]
+    if dy.dtype != torch.float32 or not dy.is_contiguous() or tuple(dy.shape) != (M, K):
+        raise ValueError("dy must be a contiguous float32 tensor of shape (M, K)")
+    L = lib()
+    need = L.twell_bwd_scratch_bytes(M, K, N, tw.T, tw.C, tw.R_cap)
+    if need == 0:
+        raise ValueError("invalid sizes for twell_ffn_bwd")
+    if scratch is None or scratch.numel() < need:
+        scratch = torch.empty(need, dtype=torch.uint8, device=x.device)
+    dx = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    dg, du, dd = (torch.empty((N, K), dtype=torch.float32, device=x.device) for _ in range(3))
+    st = L.twell_ffn_bwd(_bf16(x, "x", (M, K)), _bf16(wg_t, "wg_t", (N, K)), _bf16(wu_t, "wu_t", (N, K)),
+                         _bf16(wd, "wd", (N, K)), ctypes.byref(tw.buf), dy.data_ptr(), K, dx.data_ptr(),
+                         dg.data_ptr(), du.data_ptr(), dd.data_ptr(), scratch.data_ptr(), scratch.numel(),
+                         _stream(stream))
+    _check(st, "twell_ffn_bwd")
+    return dx, dg, du, dd
 
 
 def read_status(tw: TwellBuffers, stream=None):

@@ -172,6 +172,30 @@ twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint
                              int K, int N, twell_buf* tw, float* y, int* n_over_host, cudaStream_t stream);
 
 /*
+ * Backward pass over the hybrid activations (training; "Sparser, Faster,
+ * Lighter Transformer Language Models", §3-6 and §3-7: every product visits
+ * only the active units).  Given the TwELL + dense-row buffer `tw` of the
+ * forward (twell_gate_pack on the same x, wg_t) and the upstream gradient
+ * dy [M][K] (device fp32), writes, all device fp32 and fully overwritten:
+ *   dx    [M][K]  = sum_n du_n W_u^T[n] + dz_n W_g^T[n]
+ *   dwg_t [N][K]  = sum_m dz_{m,n} x_m,   dwu_t [N][K] = sum_m du_{m,n} x_m,
+ *   dwd   [N][K]  = sum_m h_{m,n} dy_m      (rows of inactive units are 0)
+ * with, per active (m, n): u = x_m W_u^T[n], dh = dy_m . W_d[n], h = u g,
+ * du = dh g, dz = dh u (g = ReLU(z) from TwELL or the row's dense-row slot).
+ * scratch: device, 256-byte aligned, >= twell_bwd_scratch_bytes(...) bytes
+ * (per-unit counts and offsets, and a unit-major list of 16-byte entries
+ * (row, h, du, dz): the hybrid activations transposed).  Limits: those of
+ * twell_buf_init and K <= 2560.  Launches two memsets and four kernels
+ * (count, scan, row pass, unit pass).  Asynchronous.  The sums over rows and
+ * units are taken in an order that atomics decide, so repeated calls agree to
+ * rounding, not bit for bit.
+ */
+size_t twell_bwd_scratch_bytes(int M, int K, int N, int T, int C, int R_cap);
+twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
+                           const twell_buf* tw, const float* dy, int K, float* dx, float* dwg_t, float* dwu_t,
+                           float* dwd, void* scratch, size_t scratch_bytes, cudaStream_t stream);
+
+/*
  * Synchronises `stream` and reads the buffer's device control words.
  * Returns TWELL_ERR_DEVICE_CHECK if a device status flag other than the
  * capacity flag is set, else TWELL_ERR_CAPACITY if n_over > R_cap, else
