@@ -15,11 +15,12 @@
 //   1. count   : active entries per hidden unit (atomic counts);
 //   2. scan    : exclusive prefix of the counts (one CTA) -> each unit's
 //                segment of a unit-major entry list (the hybrid transpose);
-//   3. rows    : static (row, tile group) units as in the small-batch
-//                up/down kernel; the W_u^T, W_d and W_g^T rows of every entry
-//                stream through a per-warp ring; the warp adds du W_u^T + dz
-//                W_g^T into dx (vector atomics, dx cleared first) and appends
-//                (row, h, du, dz) to the unit's segment;
+//   3. rows    : static units, each a row's group of TwELL tiles or one
+//                32-column chunk of an overflow tile (heavy rows are spread
+//                over many warps that way); the W_u^T, W_d and W_g^T rows of
+//                every entry stream through a per-warp ring; the warp adds
+//                du W_u^T + dz W_g^T into dx (vector atomics, dx cleared
+//                first) and appends (row, h, du, dz) to the unit's segment;
 //   4. units   : one warp per (unit, 256-column chunk) reads the unit's
 //                segment and the entries' x and dy chunks, and writes the
 //                chunk of the three weight-gradient rows (plain stores; units
@@ -55,8 +56,10 @@ struct BwdParams {
   int* off;            // [N + 1] start of each unit's segment
   int* fill;           // [N] entries written so far per unit
   BwdEntry* entries;   // unit-major entry list
+  const int* slot_row; // [R_cap] row of each dense-row slot
+  int r_cap;
   int stages, list_cap, tiles_per_unit;
-  int* ctrl;
+  int* ctrl;           // ctrl[kCtrlNOver]: slots in use
 };
 
 // ---------------------------------------------------------------- 1. count
@@ -123,9 +126,10 @@ __device__ __forceinline__ void dot8_f32_bf16(const float (&a)[8], const uint4& 
 }
 
 // Bytes of one warp's shared memory in the row pass: [ring: stages x (W_u^T row
-// | W_d row | W_g^T row)][list n: int x cap][list g: float x cap].
+// | W_d row | W_g^T row)][list n: int x cap][list g: float x cap][h, du, dz of
+// the listed entries: 3 x float x cap].
 __host__ __device__ constexpr size_t bwd_warp_bytes(int K, int stages, int list_cap) {
-  return ((static_cast<size_t>(stages) * 6 * K + static_cast<size_t>(list_cap) * 8) + 127) / 128 * 128;
+  return ((static_cast<size_t>(stages) * 6 * K + static_cast<size_t>(list_cap) * 20) + 127) / 128 * 128;
 }
 
 // Most warps per CTA of the row pass: eight while a lane's x, dy and dx
@@ -198,19 +202,30 @@ __device__ __forceinline__ void bwd_stream(const BwdParams& p, const WarpRing& w
       }
     }
     if (lane == 0) {
-      const int pos = p.off[n] + atomicAdd(p.fill + n, 1);
-      BwdEntry en;
-      en.m = m;
-      en.h = u * g;
-      en.du = du;
-      en.dz = dz;
-      p.entries[pos] = en;
+      float* keep = w.list_g + w.list_cap;  // h, du, dz of entry e, appended below
+      keep[e] = u * g;
+      keep[w.list_cap + e] = du;
+      keep[2 * w.list_cap + e] = dz;
     }
     // This lane has read the slot: refill it with the entry S places ahead.
     if (e + S < E) bwd_issue<KV>(p, w, slot, w.list_n[e + S], lane);
     cp_async_commit();
     slot = slot + 1 == S ? 0 : slot + 1;
   }
+  // Append the E entries to their units' segments: one atomic round trip for
+  // up to 32 entries at a time instead of one per entry.
+  __syncwarp();
+  const float* keep = w.list_g + w.list_cap;
+  for (int j = lane; j < E; j += 32) {
+    const int n = w.list_n[j];
+    BwdEntry en;
+    en.m = m;
+    en.h = keep[j];
+    en.du = keep[w.list_cap + j];
+    en.dz = keep[2 * w.list_cap + j];
+    p.entries[p.off[n] + atomicAdd(p.fill + n, 1)] = en;
+  }
+  __syncwarp();
 }
 
 template <int KV>
@@ -241,18 +256,32 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
 
   const int tpu = p.tiles_per_unit;
   const int groups = (NT + tpu - 1) / tpu;
-  const int64_t n_units = static_cast<int64_t>(p.M) * groups;
+  const int64_t n_twell = static_cast<int64_t>(p.M) * groups;  // units over TwELL tiles
+  const int chunks = p.T / 32;
+  int n_over = ld_acquire(p.ctrl + kCtrlNOver);
+  n_over = n_over < p.r_cap ? n_over : p.r_cap;
+  const int64_t n_units = n_twell + static_cast<int64_t>(n_over) * NT * chunks;  // + overflow-tile chunks
   const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   uint4 xv[KV];
   float dyv[KV][8];
   float acc[KV][8];
   for (int64_t u = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; u < n_units; u += stride) {
-    const int row = static_cast<int>(u / groups);
-    const int t0 = static_cast<int>(u - static_cast<int64_t>(row) * groups) * tpu;
-    const int t1 = t0 + tpu < NT ? t0 + tpu : NT;
-    const int c = t0 + lane < t1 ? static_cast<int>(p.counts[static_cast<int64_t>(row) * NT + t0 + lane]) : 0;
-    if (__ballot_sync(0xffffffffu, c > 0) == 0) continue;
-    const uint32_t ov = __ballot_sync(0xffffffffu, c > p.C);
+    int row, t0 = 0, t1 = 0, slot = -1, ot = 0, oq = 0;
+    if (u < n_twell) {
+      row = static_cast<int>(u / groups);
+      t0 = static_cast<int>(u - static_cast<int64_t>(row) * groups) * tpu;
+      t1 = t0 + tpu < NT ? t0 + tpu : NT;
+      const int c = t0 + lane < t1 ? static_cast<int>(p.counts[static_cast<int64_t>(row) * NT + t0 + lane]) : 0;
+      if (__ballot_sync(0xffffffffu, c > 0 && c <= p.C) == 0) continue;
+    } else {
+      const int64_t item = u - n_twell;
+      slot = static_cast<int>(item / (NT * chunks));
+      const int rem = static_cast<int>(item - static_cast<int64_t>(slot) * NT * chunks);
+      ot = rem / chunks;
+      oq = rem - ot * chunks;
+      row = p.slot_row[slot];
+      if (row < 0 || row >= p.M || p.counts[static_cast<int64_t>(row) * NT + ot] <= p.C) continue;
+    }
     const uint16_t* xr = p.x + static_cast<int64_t>(row) * p.K;
     const float* dyr = p.dy + static_cast<int64_t>(row) * p.K;
 #pragma unroll
@@ -267,39 +296,26 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
     }
-    int cursor = t0;
-    while (cursor < t1) {
-      const int E = list_entries(lp, w, row, cursor, t1, lane);
-      if (E > 0) bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
-    }
-    const int slot = ov ? p.row_slot[row] : -1;
-    if (slot >= 0) {
-      uint32_t rest = ov;
-      int E = 0;
+    if (slot < 0) {
+      int cursor = t0;
+      while (cursor < t1) {
+        const int E = list_entries(lp, w, row, cursor, t1, lane);
+        if (E > 0) bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
+      }
+    } else {
+      // Every positive gate of 32 columns of the overflow tile, in column order.
+      const int col = ot * p.T + oq * 32 + lane;
+      const float gv = p.dense_rows[static_cast<int64_t>(slot) * p.N + col];
+      const uint32_t bal = __ballot_sync(0xffffffffu, gv > 0.f);
       __syncwarp();
-      while (rest) {
-        const int t = t0 + __ffs(rest) - 1;
-        rest &= rest - 1;
-        if (E + p.T > w.list_cap) {
-          __syncwarp();
-          bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
-          E = 0;
-          __syncwarp();
-        }
-        const float* src = p.dense_rows + static_cast<int64_t>(slot) * p.N + static_cast<int64_t>(t) * p.T;
-        for (int j0 = 0; j0 < p.T; j0 += 32) {
-          const float gv = src[j0 + lane];
-          const uint32_t bal = __ballot_sync(0xffffffffu, gv > 0.f);
-          if (gv > 0.f) {
-            const int pos = E + __popc(bal & ((1u << lane) - 1u));
-            w.list_n[pos] = t * p.T + j0 + lane;
-            w.list_g[pos] = gv;
-          }
-          E += __popc(bal);
-        }
+      if (gv > 0.f) {
+        const int pos = __popc(bal & ((1u << lane) - 1u));
+        w.list_n[pos] = col;
+        w.list_g[pos] = gv;
       }
       __syncwarp();
-      if (E > 0) bwd_stream<KV>(p, w, E, row, xv, dyv, acc, lane);
+      if (bal == 0) continue;
+      bwd_stream<KV>(p, w, __popc(bal), row, xv, dyv, acc, lane);
     }
     float* dxr = p.dx + static_cast<int64_t>(row) * p.K;
 #pragma unroll

@@ -331,7 +331,7 @@ BwdLayout bwd_layout(int M, int N, int T, int C, int R_cap) {
 template <int KV>
 cudaError_t launch_bwd_rows_kv(BwdParams p, int sms, cudaStream_t s) {
   constexpr size_t kBudget = 232448;
-  const size_t list = static_cast<size_t>(kUpdownListCap) * 8 + 128;
+  const size_t list = static_cast<size_t>(kUpdownListCap) * 20 + 128;  // n, g, h, du, dz per listed entry
   int warps = bwd_max_warps<KV>(), stages = 0;
   for (; warps >= 2; --warps) {
     const size_t per_warp = kBudget / warps;
@@ -342,7 +342,8 @@ cudaError_t launch_bwd_rows_kv(BwdParams p, int sms, cudaStream_t s) {
   if (stages > 4) stages = 4;
   p.stages = stages;
   p.list_cap = kUpdownListCap;
-  // About two units per warp, each within the list and one ballot (<= 32 tiles).
+  // TwELL units: about two per warp, each within the list and one ballot
+  // (<= 32 tiles); overflow tiles are cut into 32-column units on the device.
   const int NT = p.N / p.T;
   const int64_t records = static_cast<int64_t>(p.M) * NT;
   const int64_t nw = static_cast<int64_t>(sms) * warps;
@@ -834,6 +835,8 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   p.fill = reinterpret_cast<int*>(sb + L.fill);
   p.off = reinterpret_cast<int*>(sb + L.off);
   p.entries = reinterpret_cast<BwdEntry*>(sb + L.entries);
+  p.slot_row = tw->slot_row;
+  p.r_cap = tw->R_cap;
   p.ctrl = tw->ctrl;
 
   TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // counts and fill

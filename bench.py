@@ -59,6 +59,8 @@ FLUSH_BYTES = 256 << 20
 # Small-batch workloads, timed from CUDA graphs over rotating weight copies.
 SMALL_BATCH_WORKLOADS = ("sweep_m16_k2048_n8192_p99", "sweep_m64_k2048_n8192_p99")
 SMALL_BATCH_COPIES = 4
+# Backward pass over the hybrid activations (training), timed on these.
+BACKWARD_WORKLOADS = ("m16384_k2560_n10240_p99_boost3pct", "m2048_k1536_n4096_p99_lognormal05")
 
 
 def load_peaks():
@@ -521,6 +523,74 @@ def measure_small_batch(tw, torch, dev, w, d, peaks, reps=25):
     return out
 
 
+def measure_backward(tw, torch, dev, w, d, steps, warmup, flush, peaks):
+    """twell_ffn_bwd after a synchronous gate pass: whole-call time (events,
+    L2 flushed before each call), per-kernel times, and a dense backward of
+    the same FFN with torch bf16 matmuls (cuBLAS) for context."""
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, wg, wu, wd = (to_dev(d[k]) for k in ("x", "wg_t", "wu_t", "wd"))
+    M, K, N, T, C = w.M, w.K, w.N, w.T, w.C
+    tb = tw.TwellBuffers(M, K, N, T, C, device=dev)
+    n_over = tw.gate_pack(x, wg, tb, sync=True)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    dy = torch.randn(M, K, device=dev, generator=g)
+    need = tw.lib().twell_bwd_scratch_bytes(M, K, N, T, C, tb.R_cap)
+    scratch = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def bwd():
+        return tw.ffn_bwd(x, wg, wu, wd, tb, dy, scratch)
+
+    def dense_bwd():
+        z = x @ wg.t()
+        u = x @ wu.t()
+        gg = torch.relu(z)
+        dyb = dy.to(torch.bfloat16)
+        dh = dyb @ wd.t()
+        du = dh * gg
+        dz = dh * u * (z > 0)
+        return du @ wu + dz @ wg, dz.t() @ x, du.t() @ x, (u * gg).t() @ dyb
+
+    def timed(fn, n):
+        out = []
+        for i in range(n):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            out.append(a.elapsed_time(b))
+        return sum(out) / len(out)
+
+    for _ in range(warmup):
+        bwd()
+    ms = timed(bwd, steps)
+    per = {}
+    for i in range(min(steps, 5)):
+        flush.fill_(i & 0xFF)
+        tr = tw.KernelTrace(capacity=8)
+        with tr:
+            bwd()
+        torch.cuda.synchronize()
+        for name, t in tr.times_ms():
+            per.setdefault(name, []).append(t)
+    for _ in range(2):
+        dense_bwd()
+    dense_ms = timed(dense_bwd, min(steps, 5))
+    st, _, _ = tw.read_status(tb)
+    stats = workload_stats(tb, w, T, C)
+    return {"workload": w.name, "M": M, "K": K, "N": N, "ms": ms, "tokens_per_s": M / (ms * 1e-3),
+            "n_over": n_over, "twell_entries": stats["twell_entries"], "status": st,
+            "kernels_ms": {k: sum(v) / len(v) for k, v in per.items()},
+            "torch_dense_backward_ms": dense_ms,
+            "torch_dense_backward": "bf16 torch matmuls (cuBLAS) and elementwise ops, recomputing z and u; "
+                                    "context only, not held to the y rule",
+            "speedup_vs_torch_dense": dense_ms / ms}
+
+
 def run_ncu_case(args):
     """The sparse path only, --warmup + 1 times, on one GPU: the launches an
     ncu capture selects from (no flush buffer, no dense FFN, no timing)."""
@@ -613,6 +683,14 @@ def run_native(args, rank, world, local_rank):
             small[name] = measure_small_batch(tw, torch, dev, ws, wl.generate(ws), peaks)
             torch.cuda.empty_cache()
 
+    backward = {}
+    if not args.no_extra:
+        for name in BACKWARD_WORKLOADS:
+            wb = wl.WORKLOADS[name]
+            backward[name] = measure_backward(tw, torch, dev, wb, wl.generate(wb), args.steps, args.warmup, flush,
+                                              peaks)
+            torch.cuda.empty_cache()
+
     # One collective on every rank: the job's time is the slowest rank's.
     ms, e2e_ms = max_over_ranks([head["ms_per_step"], e2e_ms], world, dev)
     if rank != 0:
@@ -651,6 +729,7 @@ def run_native(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "other_workloads": others,
         "small_batch": small,
+        "backward": backward,
     }
     print(json.dumps(line), flush=True)
 
