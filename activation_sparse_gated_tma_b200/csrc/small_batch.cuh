@@ -79,6 +79,55 @@ __device__ __forceinline__ int pack_row_tile(const float (&v)[T / 32], const Gat
   return 0;
 }
 
+// pack_row_tile for up to R rows at once (rows[r] < 0: no row), written as
+// straight-line code so that the rows' ballots, ranks and stores interleave;
+// overflow tiles (rare) then take pack_row_tile's slot path one at a time.
+template <int T, int R>
+__device__ __forceinline__ int pack_rows(const float (&v)[R][T / 32], const int (&rows)[R], const GateTwellParams& p,
+                                         int t, int lane, int* ctrl) {
+  constexpr int V = T / 32;
+  const int NT = p.N / T;
+  const uint32_t lower = (1u << lane) - 1u;
+  uint32_t act[R][V];
+  int cnt[R], off[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < V; ++j) act[r][j] = __ballot_sync(0xffffffffu, rows[r] >= 0 && v[r][j] > 0.f);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    cnt[r] = 0;
+    off[r] = 0;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      cnt[r] += __popc(act[r][j]);
+      off[r] += __popc(act[r][j] & lower);
+    }
+  }
+  int listed = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (rows[r] < 0) continue;
+    const int64_t rec = static_cast<int64_t>(rows[r]) * NT + t;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if ((act[r][j] >> lane) & 1u) {
+        if (off[r] < p.C) {
+          p.idx[rec * p.C + off[r]] = static_cast<uint8_t>(lane * V + j);
+          p.vals[rec * p.C + off[r]] = v[r][j];
+        }
+        ++off[r];
+      }
+    }
+    if (lane == 0) p.counts[rec] = static_cast<uint16_t>(cnt[r]);
+    if (cnt[r] <= p.C) listed += cnt[r];
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (rows[r] >= 0 && cnt[r] > p.C) pack_row_tile<T>(v[r], p, rows[r], t, lane, ctrl);  // slot path
+  return listed;
+}
+
 // Scratch slots per 128-unit tile: the host sizes the CTA ranges (at least a
 // third of a tile's k blocks each) so that no tile has more contributors.
 constexpr int kStreamSlots = 4;
@@ -294,17 +343,18 @@ __device__ __forceinline__ void stream_run(const CUtensorMap* tmW, const CUtenso
                               ? __ldcg(reinterpret_cast<const float4*>(base + (static_cast<int64_t>(j) * p.M + m) * 128))
                               : make_float4(0.f, 0.f, 0.f, 0.f);
               }
+            float v[4][4];
+            int rows[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-              const int m = m0 + 4 * r;
-              if (m >= p.M) break;
-              float v[4] = {a[r][0].x, a[r][0].y, a[r][0].z, a[r][0].w};
+              rows[r] = m0 + 4 * r < p.M ? m0 + 4 * r : -1;
+              v[r][0] = a[r][0].x; v[r][1] = a[r][0].y; v[r][2] = a[r][0].z; v[r][3] = a[r][0].w;
 #pragma unroll
               for (int j = 1; j < kStreamSlots; ++j) {
-                v[0] += a[r][j].x; v[1] += a[r][j].y; v[2] += a[r][j].z; v[3] += a[r][j].w;
+                v[r][0] += a[r][j].x; v[r][1] += a[r][j].y; v[r][2] += a[r][j].z; v[r][3] += a[r][j].w;
               }
-              listed += pack_row_tile<128>(v, p.pk, m, t, lane, ctrl);
             }
+            listed += pack_rows<128, 4>(v, rows, p.pk, t, lane, ctrl);
           }
         } else {
           // Lane l holds columns [8l, 8l + 8): 128-unit tile 2t + l / 16.
@@ -325,19 +375,20 @@ __device__ __forceinline__ void stream_run(const CUtensorMap* tmW, const CUtenso
                 a[r][j][0] = use ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
                 a[r][j][1] = use ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
               }
+            float v[2][8];
+            int rows[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-              const int m = m0 + 4 * r;
-              if (m >= p.M) break;
-              float v[8] = {a[r][0][0].x, a[r][0][0].y, a[r][0][0].z, a[r][0][0].w,
-                            a[r][0][1].x, a[r][0][1].y, a[r][0][1].z, a[r][0][1].w};
+              rows[r] = m0 + 4 * r < p.M ? m0 + 4 * r : -1;
+              v[r][0] = a[r][0][0].x; v[r][1] = a[r][0][0].y; v[r][2] = a[r][0][0].z; v[r][3] = a[r][0][0].w;
+              v[r][4] = a[r][0][1].x; v[r][5] = a[r][0][1].y; v[r][6] = a[r][0][1].z; v[r][7] = a[r][0][1].w;
 #pragma unroll
               for (int j = 1; j < kStreamSlots; ++j) {
-                v[0] += a[r][j][0].x; v[1] += a[r][j][0].y; v[2] += a[r][j][0].z; v[3] += a[r][j][0].w;
-                v[4] += a[r][j][1].x; v[5] += a[r][j][1].y; v[6] += a[r][j][1].z; v[7] += a[r][j][1].w;
+                v[r][0] += a[r][j][0].x; v[r][1] += a[r][j][0].y; v[r][2] += a[r][j][0].z; v[r][3] += a[r][j][0].w;
+                v[r][4] += a[r][j][1].x; v[r][5] += a[r][j][1].y; v[r][6] += a[r][j][1].z; v[r][7] += a[r][j][1].w;
               }
-              listed += pack_row_tile<256>(v, p.pk, m, t, lane, ctrl);
             }
+            listed += pack_rows<256, 2>(v, rows, p.pk, t, lane, ctrl);
           }
         }
         if (lane == 0 && listed > 0) atomicAdd(ctrl + kCtrlEntries, listed);
