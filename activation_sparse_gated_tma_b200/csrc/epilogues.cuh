@@ -337,6 +337,99 @@ struct EpiOverflowProduct {
 };
 
 // ---------------------------------------------------------------------------
+// Backward over the dense-row slots ("Sparser, Faster, Lighter Transformer
+// Language Models", §3-6: the dense backup rows take the dense tensor-core
+// path in training too).  The accumulator holds dh = dy_m W_d^T for slot r
+// (m = slot_row[r]) on 128 hidden units.  On units of the row's overflow
+// tiles with g = ReLU(z) > 0 (the stored gate) the epilogue forms, with u =
+// x_m W_u^T (fp32, from the previous GEMM),
+//   du = dh g,  dz = dh u,  h = u g
+// (0 elsewhere: TwELL tiles are served by the gather passes), and writes each
+// as bf16 hi + lo: du and dz row-major ([R][2N], hi in columns [0, N)) for the
+// dx GEMMs, and h, du, dz transposed ([N][2 R_pad], hi in columns [0, R_pad))
+// for the weight-gradient GEMMs, which reduce over the slots.
+struct EpiBwdSlots : EpiNoPrepare {
+  static constexpr int kScratchBytes = 0;
+  struct Params {
+    const float* u;           // [R][N] x_over W_u^T
+    const float* dense_rows;  // [R_cap][N] stored ReLU gates
+    const uint16_t* counts;   // [M][N/T]
+    const int* slot_row;      // [R_cap]
+    uint16_t* du_rows;        // [R][2N]
+    uint16_t* dz_rows;        // [R][2N]
+    uint16_t* h_t;            // [N][2 R_pad]
+    uint16_t* du_t;           // [N][2 R_pad]
+    uint16_t* dz_t;           // [N][2 R_pad]
+    int N, T, C, r_pad;
+  };
+  template <int BN>
+  static __device__ __forceinline__ void run(const Params& p, const Pre<BN>&, uint32_t taddr, int row, int m_rows,
+                                             int nb, int, int*, void*, int, int) {
+    const bool valid = row < m_rows;
+    const int m = valid ? p.slot_row[row] : -1;
+    const int NT = p.N / p.T;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32(taddr + c * 32, r);
+      tmem_wait_ld();
+      const int n0 = nb * BN + c * 32;
+      const bool ov = m >= 0 && p.counts[static_cast<int64_t>(m) * NT + n0 / p.T] > p.C;
+      float du[32], dz[32], h[32];
+      if (ov) {
+        const float4* u4 = reinterpret_cast<const float4*>(p.u + static_cast<int64_t>(row) * p.N + n0);
+        const float4* g4 = reinterpret_cast<const float4*>(p.dense_rows + static_cast<int64_t>(row) * p.N + n0);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const float4 uu = u4[v], gg = g4[v];
+          const float us[4] = {uu.x, uu.y, uu.z, uu.w}, gs[4] = {gg.x, gg.y, gg.z, gg.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float dh = __uint_as_float(r[4 * v + e]);
+            const bool on = gs[e] > 0.f;
+            du[4 * v + e] = on ? dh * gs[e] : 0.f;
+            dz[4 * v + e] = on ? dh * us[e] : 0.f;
+            h[4 * v + e] = on ? us[e] * gs[e] : 0.f;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) du[j] = dz[j] = h[j] = 0.f;
+      }
+      if (!valid) continue;
+      uint4* dur = reinterpret_cast<uint4*>(p.du_rows + static_cast<int64_t>(row) * 2 * p.N + n0);
+      uint4* dzr = reinterpret_cast<uint4*>(p.dz_rows + static_cast<int64_t>(row) * 2 * p.N + n0);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        float a[8], b[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          a[e] = du[8 * v + e];
+          b[e] = dz[8 * v + e];
+        }
+        split_bf16x8(a, dur[v], dur[v + p.N / 8]);
+        split_bf16x8(b, dzr[v], dzr[v + p.N / 8]);
+      }
+      // Transposed: for a fixed unit the warp's 32 rows are 32 consecutive slots.
+      const int64_t ld = 2 * static_cast<int64_t>(p.r_pad);
+#pragma unroll 4
+      for (int j = 0; j < 32; ++j) {
+        const int64_t o = static_cast<int64_t>(n0 + j) * ld + row;
+        const uint16_t hh = float_to_bf16_bits(h[j]);
+        const uint16_t uh = float_to_bf16_bits(du[j]);
+        const uint16_t zh = float_to_bf16_bits(dz[j]);
+        p.h_t[o] = hh;
+        p.h_t[o + p.r_pad] = float_to_bf16_bits(h[j] - bf16_bits_to_float(hh));
+        p.du_t[o] = uh;
+        p.du_t[o + p.r_pad] = float_to_bf16_bits(du[j] - bf16_bits_to_float(uh));
+        p.dz_t[o] = zh;
+        p.dz_t[o + p.r_pad] = float_to_bf16_bits(dz[j] - bf16_bits_to_float(zh));
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
 // Overflow path, second stage: y[slot_row[r]][col] += acc (vector atomics, so
 // split-K slices and the fused kernel's earlier partial sum combine).
 struct EpiAccumulateRows : EpiNoPrepare {

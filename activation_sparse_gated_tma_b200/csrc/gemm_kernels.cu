@@ -55,6 +55,16 @@ cudaError_t launch_gate_twell_pair(int T, const CUtensorMap& tm_x, const CUtenso
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_store_f32_kmajor(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmGeom& g,
+                                   const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s) {
+  return launch<128, false, false, 6, EpiStoreF32>(tm_a, tm_b, tm_b, g, p, ctrl, grid, s);
+}
+
+cudaError_t launch_bwd_slots(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmGeom& g,
+                             const EpiBwdSlots::Params& p, int* ctrl, int grid, cudaStream_t s) {
+  return launch<128, false, false, 6, EpiBwdSlots>(tm_a, tm_b, tm_b, g, p, ctrl, grid, s);
+}
+
 cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
                                  const GemmGeom& g, const EpiGatedProduct::Params& p, int* ctrl, int grid,
                                  cudaStream_t s) {

@@ -21,6 +21,12 @@ cudaError_t launch_gate_twell(int T, int bn, const CUtensorMap& tm_x, const CUte
 // tm_wg's box is 128 rows (each CTA's half of a tile's columns).  grid is even.
 cudaError_t launch_gate_twell_pair(int T, const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const GemmGeom& g,
                                    const GateTwellParams& p, int* ctrl, int grid, cudaStream_t s);
+// D = A B^T (both K-major), fp32 store (or vector-atomic add), BN = 128.
+cudaError_t launch_store_f32_kmajor(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmGeom& g,
+                                   const EpiStoreF32::Params& p, int* ctrl, int grid, cudaStream_t s);
+// Backward, dense-row slots: dh = [dy_hi | dy_lo] W_d^T with the du/dz/h epilogue, BN = 128.
+cudaError_t launch_bwd_slots(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmGeom& g,
+                             const EpiBwdSlots::Params& p, int* ctrl, int grid, cudaStream_t s);
 // h = (x W_u) * ReLU(x W_g), bf16, BN = 128.
 cudaError_t launch_gated_product(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
                                  const GemmGeom& g, const EpiGatedProduct::Params& p, int* ctrl, int grid,

@@ -27,6 +27,7 @@
 //                with no entry get zero rows).
 #pragma once
 
+#include "epilogues.cuh"
 #include "sparse_updown.cuh"
 
 namespace twell {
@@ -58,6 +59,7 @@ struct BwdParams {
   BwdEntry* entries;   // unit-major entry list
   const int* slot_row; // [R_cap] row of each dense-row slot
   int r_cap;
+  int gather_overflow; // 1: overflow tiles also go through the row pass (else the dense-row GEMMs)
   int stages, list_cap, tiles_per_unit;
   int* ctrl;           // ctrl[kCtrlNOver]: slots in use
 };
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(256) twell_bwd_count_kernel(const BwdParams p)
     const int t = static_cast<int>(r - static_cast<int64_t>(m) * NT);
     if (c <= p.C) {
       for (int s = 0; s < c; ++s) atomicAdd(p.cnt + t * p.T + p.idx[r * p.C + s], 1);
-    } else {
+    } else if (p.gather_overflow) {
       const int slot = p.row_slot[m];
       if (slot < 0) continue;
       const float* g = p.dense_rows + static_cast<int64_t>(slot) * p.N + static_cast<int64_t>(t) * p.T;
@@ -258,8 +260,7 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
   const int groups = (NT + tpu - 1) / tpu;
   const int64_t n_twell = static_cast<int64_t>(p.M) * groups;  // units over TwELL tiles
   const int chunks = p.T / 32;
-  int n_over = ld_acquire(p.ctrl + kCtrlNOver);
-  n_over = n_over < p.r_cap ? n_over : p.r_cap;
+  const int n_over = p.gather_overflow ? min(ld_acquire(p.ctrl + kCtrlNOver), p.r_cap) : 0;
   const int64_t n_units = n_twell + static_cast<int64_t>(n_over) * NT * chunks;  // + overflow-tile chunks
   const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   uint4 xv[KV];
@@ -326,6 +327,42 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
         atomicAdd(reinterpret_cast<float4*>(dxr + k0 + 4), make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]));
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------- 5. dense-row slots
+// Operands of the slots' backward GEMMs: for slot r < R, dy of its row split
+// into bf16 hi + lo ([R_pad][2K] and the halves [R_pad][K] apart) and its x
+// row ([R_pad][K]); rows R .. R_pad - 1 are zero, so the GEMMs that reduce
+// over slots may run over R_pad.
+__global__ void __launch_bounds__(256) twell_bwd_slot_operands_kernel(const float* __restrict__ dy,
+                                                                       const uint16_t* __restrict__ x_over,
+                                                                       const int* __restrict__ slot_row, int R,
+                                                                       int r_pad, int K, uint16_t* dy_cat,
+                                                                       uint16_t* dy_hi, uint16_t* dy_lo,
+                                                                       uint16_t* x_pad) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int per_row = K / 8;
+  const int64_t items = static_cast<int64_t>(r_pad) * per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < items;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / per_row);
+    const int k = static_cast<int>(i - static_cast<int64_t>(r) * per_row) * 8;
+    uint4 hi = make_uint4(0, 0, 0, 0), lo = hi, xv = hi;
+    if (r < R) {
+      const int m = slot_row[r];
+      const float4 a = *reinterpret_cast<const float4*>(dy + static_cast<int64_t>(m) * K + k);
+      const float4 b = *reinterpret_cast<const float4*>(dy + static_cast<int64_t>(m) * K + k + 4);
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      split_bf16x8(v, hi, lo);
+      xv = *reinterpret_cast<const uint4*>(x_over + static_cast<int64_t>(r) * K + k);
+    }
+    *reinterpret_cast<uint4*>(dy_cat + static_cast<int64_t>(r) * 2 * K + k) = hi;
+    *reinterpret_cast<uint4*>(dy_cat + static_cast<int64_t>(r) * 2 * K + K + k) = lo;
+    *reinterpret_cast<uint4*>(dy_hi + static_cast<int64_t>(r) * K + k) = hi;
+    *reinterpret_cast<uint4*>(dy_lo + static_cast<int64_t>(r) * K + k) = lo;
+    *reinterpret_cast<uint4*>(x_pad + static_cast<int64_t>(r) * K + k) = xv;
   }
 }
 

@@ -309,21 +309,38 @@ cudaError_t launch_fused_small(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
 }
 
 // ---------------------------------------------------------------- backward
-constexpr int kBwdMaxK = 2560;  // the row pass keeps x, dy and dx pieces of a row in registers
+constexpr int kBwdMaxK = 2560;      // the row pass keeps x, dy and dx pieces of a row in registers
+constexpr int kBwdGatherSlots = 8;  // up to this many slotted rows go through the gather passes
 
 struct BwdLayout {
-  size_t cnt, fill, off, entries, total;
+  size_t cnt, fill, off, entries;
+  // dense-row slots (R_pad = R_cap rounded up to 64)
+  size_t dy_cat, dy_hi, dy_lo, x_pad, u, du_rows, dz_rows, h_t, du_t, dz_t;
+  size_t total;
   int64_t cap;
+  int r_pad_max;
 };
 
-BwdLayout bwd_layout(int M, int N, int T, int C, int R_cap) {
+BwdLayout bwd_layout(int M, int K, int N, int T, int C, int R_cap) {
   BwdLayout L;
   L.cap = static_cast<int64_t>(M) * (N / T) * C + static_cast<int64_t>(R_cap) * N;
+  L.r_pad_max = (R_cap + 63) / 64 * 64;
+  const size_t rp = static_cast<size_t>(L.r_pad_max);
   size_t o = 0;
   L.cnt = o; o = align256(o + size_t(N) * 4);
   L.fill = o; o = align256(o + size_t(N) * 4);
   L.off = o; o = align256(o + size_t(N + 1) * 4);
   L.entries = o; o = align256(o + size_t(L.cap) * sizeof(BwdEntry));
+  L.dy_cat = o; o = align256(o + rp * 2 * K * 2);
+  L.dy_hi = o; o = align256(o + rp * K * 2);
+  L.dy_lo = o; o = align256(o + rp * K * 2);
+  L.x_pad = o; o = align256(o + rp * K * 2);
+  L.u = o; o = align256(o + rp * N * 4);
+  L.du_rows = o; o = align256(o + rp * 2 * N * 2);
+  L.dz_rows = o; o = align256(o + rp * 2 * N * 2);
+  L.h_t = o; o = align256(o + size_t(N) * 2 * rp * 2);
+  L.du_t = o; o = align256(o + size_t(N) * 2 * rp * 2);
+  L.dz_t = o; o = align256(o + size_t(N) * 2 * rp * 2);
   L.total = o;
   return L;
 }
@@ -804,7 +821,7 @@ twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint
 
 size_t twell_bwd_scratch_bytes(int M, int K, int N, int T, int C, int R_cap) {
   if (!shape_ok(M, K, N, T, C, R_cap)) return 0;
-  return bwd_layout(M, N, T, C, R_cap).total;
+  return bwd_layout(M, K, N, T, C, R_cap).total;
 }
 
 twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
@@ -818,18 +835,28 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   if (!aligned16(x) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(dy) || !aligned16(dx) ||
       !aligned16(dwg_t) || !aligned16(dwu_t) || !aligned16(dwd))
     return fail(TWELL_ERR_INVALID, "every array must be non-NULL and 16-byte aligned");
-  const BwdLayout L = bwd_layout(tw->M, tw->N, tw->T, tw->C, tw->R_cap);
+  const int M = tw->M, N = tw->N;
+  const BwdLayout L = bwd_layout(M, K, N, tw->T, tw->C, tw->R_cap);
   if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u))
     return fail(TWELL_ERR_INVALID, "scratch must be non-NULL and 256-byte aligned");
   if (scratch_bytes < L.total) return fail(TWELL_ERR_INVALID, "scratch too small: %zu < %zu bytes", scratch_bytes, L.total);
   DeviceInfo dev;
   if ((st = device_info(dev)) != TWELL_OK) return st;
 
+  // The number of slotted rows sizes the dense-row GEMMs: read it once.
+  int n_over = 0;
+  TW_CUDA(cudaMemcpyAsync(&n_over, tw->ctrl + kCtrlNOver, sizeof n_over, cudaMemcpyDeviceToHost, stream));
+  TW_CUDA(cudaStreamSynchronize(stream));
+  const int R = n_over < tw->R_cap ? n_over : tw->R_cap;
+  // A handful of slotted rows is cheaper through the gather passes than
+  // through eight GEMM launches.
+  const bool dense_slots = R > kBwdGatherSlots;
+
   uint8_t* sb = static_cast<uint8_t*>(scratch);
   BwdParams p = {};
   p.x = x; p.wg_t = wg_t; p.wu_t = wu_t; p.wd = wd; p.dy = dy;
   p.counts = tw->counts; p.idx = tw->idx; p.vals = tw->vals; p.row_slot = tw->row_slot; p.dense_rows = tw->dense_rows;
-  p.M = tw->M; p.K = K; p.N = tw->N; p.T = tw->T; p.C = tw->C;
+  p.M = M; p.K = K; p.N = N; p.T = tw->T; p.C = tw->C;
   p.dx = dx; p.dwg_t = dwg_t; p.dwu_t = dwu_t; p.dwd = dwd;
   p.cnt = reinterpret_cast<int*>(sb + L.cnt);
   p.fill = reinterpret_cast<int*>(sb + L.fill);
@@ -837,11 +864,12 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   p.entries = reinterpret_cast<BwdEntry*>(sb + L.entries);
   p.slot_row = tw->slot_row;
   p.r_cap = tw->R_cap;
+  p.gather_overflow = dense_slots ? 0 : 1;
   p.ctrl = tw->ctrl;
 
   TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // counts and fill
-  TW_CUDA(cudaMemsetAsync(dx, 0, static_cast<size_t>(tw->M) * K * sizeof(float), stream));
-  const int64_t records = static_cast<int64_t>(tw->M) * (tw->N / tw->T);
+  TW_CUDA(cudaMemsetAsync(dx, 0, static_cast<size_t>(M) * K * sizeof(float), stream));
+  const int64_t records = static_cast<int64_t>(M) * (N / tw->T);
   const int64_t cgrid = (records + 255) / 256;
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_pdl(twell_bwd_count_kernel, static_cast<int>(cgrid < 4 * dev.sms ? cgrid : 4 * dev.sms), 256, 0,
@@ -853,12 +881,89 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_bwd_rows(p, dev.sms, stream));
   TW_CUDA(trace_end(stream, "bwd_rows"));
-  const int64_t items = static_cast<int64_t>(tw->N) * ((K + 255) / 256);
+  const int64_t items = static_cast<int64_t>(N) * ((K + 255) / 256);
   const int64_t ugrid = (items + 7) / 8;
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_pdl(twell_bwd_units_kernel, static_cast<int>(ugrid < 8 * dev.sms ? ugrid : 8 * dev.sms), 256, 0,
                      stream, p));
   TW_CUDA(trace_end(stream, "bwd_units"));
+  if (!dense_slots) return TWELL_OK;
+
+  // ---- dense-row slots on the tensor cores (after the unit pass: the weight
+  // gradients are added into the rows it wrote).
+  const int r_pad = (R + 63) / 64 * 64;
+  uint16_t* dy_cat = reinterpret_cast<uint16_t*>(sb + L.dy_cat);
+  uint16_t* dy_hi = reinterpret_cast<uint16_t*>(sb + L.dy_hi);
+  uint16_t* dy_lo = reinterpret_cast<uint16_t*>(sb + L.dy_lo);
+  uint16_t* x_pad = reinterpret_cast<uint16_t*>(sb + L.x_pad);
+  float* u = reinterpret_cast<float*>(sb + L.u);
+  uint16_t* du_rows = reinterpret_cast<uint16_t*>(sb + L.du_rows);
+  uint16_t* dz_rows = reinterpret_cast<uint16_t*>(sb + L.dz_rows);
+  uint16_t* h_t = reinterpret_cast<uint16_t*>(sb + L.h_t);
+  uint16_t* du_t = reinterpret_cast<uint16_t*>(sb + L.du_t);
+  uint16_t* dz_t = reinterpret_cast<uint16_t*>(sb + L.dz_t);
+  const size_t t_bytes = static_cast<size_t>(N) * 2 * r_pad * 2;
+  TW_CUDA(cudaMemsetAsync(h_t, 0, t_bytes, stream));
+  TW_CUDA(cudaMemsetAsync(du_t, 0, t_bytes, stream));
+  TW_CUDA(cudaMemsetAsync(dz_t, 0, t_bytes, stream));
+  const int64_t oitems = static_cast<int64_t>(r_pad) * (K / 8);
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_pdl(twell_bwd_slot_operands_kernel, static_cast<int>((oitems + 255) / 256), 256, 0, stream, dy,
+                     tw->x_over, tw->slot_row, R, r_pad, K, dy_cat, dy_hi, dy_lo, x_pad));
+  TW_CUDA(trace_end(stream, "bwd_slot_operands"));
+
+  CUtensorMap tm_xpad, tm_wu_k, tm_dycat, tm_wd_k, tm_du_rows, tm_dz_rows, tm_wu_mn, tm_wg_mn, tm_du_t, tm_dz_t,
+      tm_h_t, tm_xpad_mn, tm_dyhi_mn, tm_dylo_mn;
+  if ((st = tmap_bf16(x_pad, K, r_pad, kBM, tm_xpad)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wu_t, K, N, 128, tm_wu_k)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(dy_cat, 2 * K, r_pad, kBM, tm_dycat)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wd, K, N, 128, tm_wd_k)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(du_rows, 2 * N, r_pad, kBM, tm_du_rows)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(dz_rows, 2 * N, r_pad, kBM, tm_dz_rows)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wu_t, K, N, 64, tm_wu_mn)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(wg_t, K, N, 64, tm_wg_mn)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(du_t, 2 * r_pad, N, kBM, tm_du_t)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(dz_t, 2 * r_pad, N, kBM, tm_dz_t)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(h_t, 2 * r_pad, N, kBM, tm_h_t)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(x_pad, K, r_pad, 64, tm_xpad_mn)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(dy_hi, K, r_pad, 64, tm_dyhi_mn)) != TWELL_OK) return st;
+  if ((st = tmap_bf16(dy_lo, K, r_pad, 64, tm_dylo_mn)) != TWELL_OK) return st;
+
+  // u = x_slot W_u^T  [R][N] fp32
+  EpiStoreF32::Params pu{u, N, N, 0};
+  GemmGeom gu{R, N, K, nullptr, kGateGroupM, 0, 1};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_store_f32_kmajor(tm_xpad, tm_wu_k, gu, pu, tw->ctrl, gemm_grid(R, N, 128, dev.sms), stream));
+  TW_CUDA(trace_end(stream, "bwd_slot_u"));
+  // dh = [dy_hi | dy_lo] W_d^T, epilogue: du, dz, h on the overflow tiles
+  EpiBwdSlots::Params ps;
+  ps.u = u; ps.dense_rows = tw->dense_rows; ps.counts = tw->counts; ps.slot_row = tw->slot_row;
+  ps.du_rows = du_rows; ps.dz_rows = dz_rows; ps.h_t = h_t; ps.du_t = du_t; ps.dz_t = dz_t;
+  ps.N = N; ps.T = tw->T; ps.C = tw->C; ps.r_pad = r_pad;
+  GemmGeom gh{R, N, 2 * K, nullptr, kGateGroupM, K / kBK, 1};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_bwd_slots(tm_dycat, tm_wd_k, gh, ps, tw->ctrl, gemm_grid(R, N, 128, dev.sms), stream));
+  TW_CUDA(trace_end(stream, "bwd_slot_dh"));
+  // dx[slot rows] += [du_hi | du_lo] W_u^T... as rows of W_u^T: sum_n du_n wu_t[n]; likewise dz with W_g^T
+  const int ksx = choose_k_splits(R, K, 256, 2 * N, dev.sms);
+  EpiAccumulateRows::Params px{dx, tw->slot_row, K, K};
+  GemmGeom gx{R, K, 2 * N, nullptr, kGateGroupM, N / kBK, ksx};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_overflow_down(tm_du_rows, tm_wu_mn, gx, px, tw->ctrl, gemm_grid(R, K, 256, dev.sms, ksx), stream));
+  TW_CUDA(launch_overflow_down(tm_dz_rows, tm_wg_mn, gx, px, tw->ctrl, gemm_grid(R, K, 256, dev.sms, ksx), stream));
+  TW_CUDA(trace_end(stream, "bwd_slot_dx"));
+  // dW += (per-slot factor)^T (slot rows): reductions over the R_pad slots
+  const int ksw = choose_k_splits(N, K, 256, 2 * r_pad, dev.sms);
+  GemmGeom gw{N, K, 2 * r_pad, nullptr, kGateGroupM, r_pad / kBK, ksw};
+  const int wgrid = gemm_grid(N, K, 256, dev.sms, ksw);
+  EpiStoreF32::Params pwu{dwu_t, K, K, 1}, pwg{dwg_t, K, K, 1}, pwd{dwd, K, K, 1};
+  TW_CUDA(trace_begin(stream));
+  TW_CUDA(launch_down_store(tm_du_t, tm_xpad_mn, gw, pwu, tw->ctrl, wgrid, stream));
+  TW_CUDA(launch_down_store(tm_dz_t, tm_xpad_mn, gw, pwg, tw->ctrl, wgrid, stream));
+  TW_CUDA(launch_down_store(tm_h_t, tm_dyhi_mn, gw, pwd, tw->ctrl, wgrid, stream));
+  TW_CUDA(launch_down_store(tm_h_t, tm_dylo_mn, gw, pwd, tw->ctrl, wgrid, stream));
+  TW_CUDA(trace_end(stream, "bwd_slot_dw"));
+  g_launches += 4;  // the brackets above hold two dx and four weight-gradient launches
   return TWELL_OK;
 }
 
