@@ -11,13 +11,14 @@
 //   dx += du W_u^T[n] + dz W_g^T[n]
 //   dW_d[n] += h dy,  dW_u^T[n] += du x,  dW_g^T[n] += dz x
 //
-// Three passes:
+// Passes:
 //   1. count   : active entries per hidden unit (atomic counts);
 //   2. scan    : exclusive prefix of the counts (one CTA) -> each unit's
 //                segment of a unit-major entry list (the hybrid transpose);
-//   3. rows    : static units, each a row's group of TwELL tiles or one
-//                32-column chunk of an overflow tile (heavy rows are spread
-//                over many warps that way); the W_u^T, W_d and W_g^T rows of
+//   3. rows    : static units: a row's TwELL entries cut into shares of at
+//                most 32 entries (by tile ranges, from a per-row count and
+//                a scan of the units per row), or, when only a few rows hold
+//                dense-row slots, one 32-column chunk of an overflow tile; the W_u^T, W_d and W_g^T rows of
 //                every entry stream through a per-warp ring; the warp adds
 //                du W_u^T + dz W_g^T into dx (vector atomics, dx cleared
 //                first) and appends (row, h, du, dz) to the unit's segment;
@@ -60,7 +61,9 @@ struct BwdParams {
   const int* slot_row; // [R_cap] row of each dense-row slot
   int r_cap;
   int gather_overflow; // 1: overflow tiles also go through the row pass (else the dense-row GEMMs)
-  int stages, list_cap, tiles_per_unit;
+  int* row_entries;    // [M] TwELL entries per row
+  int* row_units;      // [M + 1] first row-pass unit of each row (exclusive prefix)
+  int stages, list_cap;
   int* ctrl;           // ctrl[kCtrlNOver]: slots in use
 };
 
@@ -78,6 +81,7 @@ __global__ void __launch_bounds__(256) twell_bwd_count_kernel(const BwdParams p)
     const int t = static_cast<int>(r - static_cast<int64_t>(m) * NT);
     if (c <= p.C) {
       for (int s = 0; s < c; ++s) atomicAdd(p.cnt + t * p.T + p.idx[r * p.C + s], 1);
+      atomicAdd(p.row_entries + m, c);
     } else if (p.gather_overflow) {
       const int slot = p.row_slot[m];
       if (slot < 0) continue;
@@ -89,17 +93,27 @@ __global__ void __launch_bounds__(256) twell_bwd_count_kernel(const BwdParams p)
 }
 
 // ---------------------------------------------------------------- 2. scan
-// One CTA of 1024 threads: thread i sums its run of consecutive counts, the
-// CTA scans the 1024 sums, and each thread writes its run's offsets.
-__global__ void __launch_bounds__(1024) twell_bwd_scan_kernel(const BwdParams p) {
+// One CTA of 1024 threads, exclusive prefix of n values: thread i sums its
+// run of consecutive values, the CTA scans the 1024 sums, and each thread
+// writes its run's offsets; out[n] is the total.  mode 0: the values are
+// in[i]; mode 1: the row-pass units of row i, ceil(in[i] / kBwdUnitEntries).
+constexpr int kBwdUnitEntries = 32;  // row-pass unit: at most this many TwELL entries
+
+__device__ __forceinline__ int bwd_scan_value(const int* in, int i, int mode) {
+  const int v = in[i];
+  return mode == 0 ? v : (v + kBwdUnitEntries - 1) / kBwdUnitEntries;
+}
+
+__global__ void __launch_bounds__(1024) twell_bwd_scan_kernel(const int* __restrict__ in, int* __restrict__ out, int n,
+                                                              int mode) {
   __shared__ int part[1024];
   griddep_launch_dependents();
   griddep_wait();
-  const int per = (p.N + 1023) / 1024;
+  const int per = (n + 1023) / 1024;
   const int a = threadIdx.x * per;
-  const int b = a + per < p.N ? a + per : p.N;
+  const int b = a + per < n ? a + per : n;
   int s = 0;
-  for (int n = a; n < b; ++n) s += p.cnt[n];
+  for (int i = a; i < b; ++i) s += bwd_scan_value(in, i, mode);
   part[threadIdx.x] = s;
   __syncthreads();
   for (int o = 1; o < 1024; o <<= 1) {
@@ -109,11 +123,11 @@ __global__ void __launch_bounds__(1024) twell_bwd_scan_kernel(const BwdParams p)
     __syncthreads();
   }
   int run = part[threadIdx.x] - s;  // exclusive start of this thread's run
-  for (int n = a; n < b; ++n) {
-    p.off[n] = run;
-    run += p.cnt[n];
+  for (int i = a; i < b; ++i) {
+    out[i] = run;
+    run += bwd_scan_value(in, i, mode);
   }
-  if (threadIdx.x == 1023) p.off[p.N] = part[1023];
+  if (threadIdx.x == 1023) out[n] = part[1023];
 }
 
 // ---------------------------------------------------------------- 3. rows
@@ -256,9 +270,7 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
   lp.T = p.T;
   lp.C = p.C;
 
-  const int tpu = p.tiles_per_unit;
-  const int groups = (NT + tpu - 1) / tpu;
-  const int64_t n_twell = static_cast<int64_t>(p.M) * groups;  // units over TwELL tiles
+  const int64_t n_twell = p.row_units[p.M];  // units over TwELL tiles (rows cut by entries)
   const int chunks = p.T / 32;
   const int n_over = p.gather_overflow ? min(ld_acquire(p.ctrl + kCtrlNOver), p.r_cap) : 0;
   const int64_t n_units = n_twell + static_cast<int64_t>(n_over) * NT * chunks;  // + overflow-tile chunks
@@ -269,11 +281,31 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
   for (int64_t u = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x; u < n_units; u += stride) {
     int row, t0 = 0, t1 = 0, slot = -1, ot = 0, oq = 0;
     if (u < n_twell) {
-      row = static_cast<int>(u / groups);
-      t0 = static_cast<int>(u - static_cast<int64_t>(row) * groups) * tpu;
-      t1 = t0 + tpu < NT ? t0 + tpu : NT;
-      const int c = t0 + lane < t1 ? static_cast<int>(p.counts[static_cast<int64_t>(row) * NT + t0 + lane]) : 0;
-      if (__ballot_sync(0xffffffffu, c > 0 && c <= p.C) == 0) continue;
+      // The row whose units hold u (largest row with row_units[row] <= u).
+      int lo = 0, hi = p.M - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.row_units[mid] <= u) lo = mid; else hi = mid - 1;
+      }
+      row = lo;
+      const int k = static_cast<int>(u - p.row_units[row]);
+      const int nunits = p.row_units[row + 1] - p.row_units[row];
+      // Inclusive per-tile prefix of the row's TwELL entries (list_n as scratch),
+      // then this unit's tiles: equal shares of the row's entries.
+      const uint16_t* crow = p.counts + static_cast<int64_t>(row) * NT;
+      int total = 0;
+      __syncwarp();
+      for (int tb = 0; tb < NT; tb += 32) {
+        const int t = tb + lane;
+        const int c = t < NT ? static_cast<int>(crow[t]) : 0;
+        const int incl = warp_inclusive_scan(c > 0 && c <= p.C ? c : 0, lane);
+        if (t < NT) w.list_n[t] = total + incl;
+        total += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      __syncwarp();
+      t0 = unit_cut(w.list_n, NT, total, nunits, k);
+      t1 = unit_cut(w.list_n, NT, total, nunits, k + 1);
+      if (t0 >= t1) continue;
     } else {
       const int64_t item = u - n_twell;
       slot = static_cast<int>(item / (NT * chunks));

@@ -313,7 +313,7 @@ constexpr int kBwdMaxK = 2560;      // the row pass keeps x, dy and dx pieces of
 constexpr int kBwdGatherSlots = 8;  // up to this many slotted rows go through the gather passes
 
 struct BwdLayout {
-  size_t cnt, fill, off, entries;
+  size_t cnt, fill, row_entries, off, row_units, entries;
   // dense-row slots (R_pad = R_cap rounded up to 64)
   size_t dy_cat, dy_hi, dy_lo, x_pad, u, du_rows, dz_rows, h_t, du_t, dz_t;
   size_t total;
@@ -329,7 +329,9 @@ BwdLayout bwd_layout(int M, int K, int N, int T, int C, int R_cap) {
   size_t o = 0;
   L.cnt = o; o = align256(o + size_t(N) * 4);
   L.fill = o; o = align256(o + size_t(N) * 4);
+  L.row_entries = o; o = align256(o + size_t(M) * 4);
   L.off = o; o = align256(o + size_t(N + 1) * 4);
+  L.row_units = o; o = align256(o + size_t(M + 1) * 4);
   L.entries = o; o = align256(o + size_t(L.cap) * sizeof(BwdEntry));
   L.dy_cat = o; o = align256(o + rp * 2 * K * 2);
   L.dy_hi = o; o = align256(o + rp * K * 2);
@@ -359,14 +361,6 @@ cudaError_t launch_bwd_rows_kv(BwdParams p, int sms, cudaStream_t s) {
   if (stages > 4) stages = 4;
   p.stages = stages;
   p.list_cap = kUpdownListCap;
-  // TwELL units: about two per warp, each within the list and one ballot
-  // (<= 32 tiles); overflow tiles are cut into 32-column units on the device.
-  const int NT = p.N / p.T;
-  const int64_t records = static_cast<int64_t>(p.M) * NT;
-  const int64_t nw = static_cast<int64_t>(sms) * warps;
-  int tpu = static_cast<int>((records + 2 * nw - 1) / (2 * nw));
-  const int tpu_max = kUpdownListCap / p.C < 32 ? kUpdownListCap / p.C : 32;
-  p.tiles_per_unit = tpu < 1 ? 1 : (tpu > tpu_max ? tpu_max : tpu);
   const size_t smem = static_cast<size_t>(warps) * bwd_warp_bytes(p.K, stages, kUpdownListCap);
   cudaError_t e = cudaFuncSetAttribute(twell_bwd_rows_kernel<KV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -860,14 +854,16 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   p.dx = dx; p.dwg_t = dwg_t; p.dwu_t = dwu_t; p.dwd = dwd;
   p.cnt = reinterpret_cast<int*>(sb + L.cnt);
   p.fill = reinterpret_cast<int*>(sb + L.fill);
+  p.row_entries = reinterpret_cast<int*>(sb + L.row_entries);
   p.off = reinterpret_cast<int*>(sb + L.off);
+  p.row_units = reinterpret_cast<int*>(sb + L.row_units);
   p.entries = reinterpret_cast<BwdEntry*>(sb + L.entries);
   p.slot_row = tw->slot_row;
   p.r_cap = tw->R_cap;
   p.gather_overflow = dense_slots ? 0 : 1;
   p.ctrl = tw->ctrl;
 
-  TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // counts and fill
+  TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // unit counts, fill, row entries
   TW_CUDA(cudaMemsetAsync(dx, 0, static_cast<size_t>(M) * K * sizeof(float), stream));
   const int64_t records = static_cast<int64_t>(M) * (N / tw->T);
   const int64_t cgrid = (records + 255) / 256;
@@ -876,8 +872,11 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
                      stream, p));
   TW_CUDA(trace_end(stream, "bwd_count"));
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, p));
+  TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, static_cast<const int*>(p.cnt), p.off, N, 0));
+  TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, static_cast<const int*>(p.row_entries), p.row_units,
+                     M, 1));
   TW_CUDA(trace_end(stream, "bwd_scan"));
+  ++g_launches;  // the bracket holds two scans
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_bwd_rows(p, dev.sms, stream));
   TW_CUDA(trace_end(stream, "bwd_rows"));
