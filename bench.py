@@ -286,7 +286,7 @@ def path_roofline(M, K, N, T, C, U, R, peaks, ms):
     NT = N // T
     flops = 2.0 * M * K * N
     b_alg = 2.0 * K * N + 4.0 * K * U + 2.0 * M * K + 4.0 * M * K + 2.0 * M * NT * (2 + 3 * C) + 4.0 * R * N
-    # This build stores TwELL values and the dense-row gates in fp32: 5 bytes per slot, 4 per gate.
+    # The library stores TwELL values and the dense-row gates in fp32: 5 bytes per slot, 4 per gate.
     b_build = 2.0 * K * N + 4.0 * K * U + 2.0 * M * K + 4.0 * M * K + 2.0 * M * NT * (2 + 5 * C) + 8.0 * R * N
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = b_alg / (peaks["hbm_gbs"] * 1e9)
