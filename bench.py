@@ -603,8 +603,13 @@ def run_ncu_case(args):
     dev = {k: torch.from_numpy(d[k].view(np.int16)).view(torch.bfloat16).cuda() for k in ("x", "wg_t", "wu_t", "wd")}
     tb = tw.TwellBuffers(w.M, w.K, w.N, w.T, w.C)
     y = torch.empty(w.M, w.K, dtype=torch.float32, device="cuda")
+    dy = torch.randn(w.M, w.K, device="cuda") if args.ncu_backward else None
+    if args.ncu_backward:
+        tw.gate_pack(dev["x"], dev["wg_t"], tb, sync=True)
     for _ in range(args.warmup + 1):
-        if args.ncu_fused:
+        if args.ncu_backward:
+            tw.ffn_bwd(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"], tb, dy)
+        elif args.ncu_fused:
             tw.ffn_fused(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"], tb, y)
         else:
             tw.gate_pack(dev["x"], dev["wg_t"], tb)
@@ -613,7 +618,27 @@ def run_ncu_case(args):
     if st != tw.OK:
         raise RuntimeError(f"status {st} (n_over {n_over}, flags {flags})")
     print(json.dumps({"ncu_case": w.name, "passes": args.warmup + 1, "n_over": n_over,
-                      "call": "twell_ffn_fused" if args.ncu_fused else "twell_gate_pack + twell_ffn_fwd"}))
+                      "call": "twell_ffn_bwd" if args.ncu_backward else
+                      ("twell_ffn_fused" if args.ncu_fused else "twell_gate_pack + twell_ffn_fwd")}))
+
+
+def run_sweep(args):
+    """One JSON line per sweep workload, on one GPU, timed as the small-batch
+    block (CUDA graph over rotating weight copies)."""
+    import torch
+
+    from activation_sparse_gated_tma_b200 import twell as tw
+
+    peaks, _ = load_peaks()
+    dev = torch.device("cuda", 0)
+    for name in sorted(n for n in wl.WORKLOADS if n.startswith("sweep_")):
+        w = wl.WORKLOADS[name]
+        r = measure_small_batch(tw, torch, dev, w, wl.generate(w), peaks)
+        print(json.dumps({"sweep": name, "M": w.M, "fused_ms": r["fused"]["ms_per_step"],
+                          "two_call_ms": r["two_call"]["ms_per_step"], "dense_ms": r["dense"]["ms_per_step"],
+                          "dense_bf16h_ms": r["dense_bf16h"]["ms_per_step"], "speedup_vs_dense": r["speedup_vs_dense"],
+                          "path_roofline_frac": r["path_roofline"]["frac"], "n_over": r["n_over"]}), flush=True)
+        torch.cuda.empty_cache()
 
 
 def run_native(args, rank, world, local_rank):
@@ -746,6 +771,11 @@ def main():
     ap.add_argument("--ncu-case", action="store_true",
                     help="no timing: --warmup + 1 passes of the sparse path on --workload (for ncu captures)")
     ap.add_argument("--ncu-fused", action="store_true", help="with --ncu-case: the passes call twell_ffn_fused")
+    ap.add_argument("--ncu-backward", action="store_true",
+                    help="with --ncu-case: one synchronous gate pass, then the passes call twell_ffn_bwd")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print one JSON line per sweep workload (M 16..4096, 90/99/99.9%% sparsity), timed "
+                         "like the small-batch block, instead of the bench line")
     args = ap.parse_args()
     if args.warmup < 3 and not args.ncu_case:
         ap.error("--warmup must be >= 3")
@@ -761,6 +791,9 @@ def main():
         return
     if args.ncu_case:
         run_ncu_case(args)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
 
     import datetime
