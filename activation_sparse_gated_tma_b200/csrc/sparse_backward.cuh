@@ -206,7 +206,6 @@ __device__ __forceinline__ void bwd_stream(const BwdParams& p, const WarpRing& w
       u += __shfl_xor_sync(0xffffffffu, u, o);
       dh += __shfl_xor_sync(0xffffffffu, dh, o);
     }
-    const int n = w.list_n[e];
     const float g = w.list_g[e];
     const float du = dh * g;
     const float dz = dh * u;
