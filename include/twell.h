@@ -146,8 +146,8 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
  * Transformer Language Models", §3-5; filled by twell_gate_pack on the same
  * stream), then the dense-row path for overflow tiles (§3-6, §4-3).  wu_t, wd [N][K]
  * device bf16; y [M][K] device fp32, fully overwritten.  K must equal tw->K.
- * For M <= TWELL_SMALL_M: y is cleared (a memset on `stream`) and one
- * static-unit kernel serves TwELL and overflow tiles.  Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
+ * For M <= 256: y is cleared (a memset on `stream`) and one static-unit
+ * kernel serves TwELL and overflow tiles (no dense-row GEMMs).  Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
  * -2 in row_slot miss their overflow tiles and twell_read_status returns
  * TWELL_ERR_CAPACITY.
  */

@@ -49,7 +49,8 @@ def test_buf_init_layout_is_aligned_and_disjoint():
     NT = N // T
     spans = [("ctrl", 64 * 4), ("counts", M * NT * 2), ("idx", M * NT * C), ("vals", M * NT * C * 4),
              ("row_slot", M * 4), ("slot_row", R * 4), ("dense_rows", R * N * 4), ("x_over", R * K * 2),
-             ("h_over", R * N * 4), ("units", M * NT * 16), ("z", M * N * 4)]  # z: M <= TWELL_SMALL_M
+             ("h_over", R * N * 4), ("units", M * NT * 16),
+             ("z", 4 * M * N * 4 + NT * 4)]  # z (M <= TWELL_SMALL_M): 4 partial-sum slots, then the tile tickets
     ranges = []
     for name, size in spans:
         p = getattr(b, name)
