@@ -101,12 +101,11 @@ typedef struct twell_buf {
   int M, K, N, T, C, R_cap;
 } twell_buf;
 
-/* Batches of at most this many rows take the small-batch path.  The gate pass
+/* Batches of at most this many rows take the small-batch gate pass: it
  * streams W_g through the tensor cores with the tokens on the narrow side of
  * the tile (128 hidden units x up to 128 tokens), cut into equal contiguous
- * k ranges per SM; the last CTA to finish a TwELL tile packs it.  The up/down
- * pass splits the work statically into (row, tile group) units, one kernel for
- * TwELL and overflow tiles alike (no dense-row GEMMs). */
+ * k ranges per SM; the last CTA to finish a TwELL tile packs it.  (Batches of
+ * up to 256 rows also take the static-unit up/down pass of twell_ffn_fwd.) */
 #define TWELL_SMALL_M 128
 
 /* Bytes of device memory twell_buf_init needs for these sizes (0 if invalid). */
