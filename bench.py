@@ -210,6 +210,17 @@ def cpu_oracle_rate(d, w, rows_target_s: float, min_rows: int = 8):
     return rows.size / dt, int(rows.size), dt, nthreads
 
 
+def cpu_dense_oracle_rate(d, w, rows: int = 32):
+    """Time the fp64 oracle's dense FFN (every hidden unit) on a small row
+    sample; returns (tokens/s, rows, seconds)."""
+    import oracle
+    sample = wl.subsample_rows(w.M, min(rows, w.M), seed=8)
+    t0 = time.perf_counter()
+    oracle.ffn_dense(d["x"], d["wg_t"], d["wu_t"], d["wd"], rows=sample)
+    dt = time.perf_counter() - t0
+    return sample.size / dt, int(sample.size), dt
+
+
 # ----------------------------------------------------------------------------- ranks
 def max_over_ranks(values, world: int, device=None):
     """Element-wise maximum of per-rank timings over all ranks (one all-reduce;
@@ -277,7 +288,7 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def path_roofline(M, K, N, T, C, U, R, peaks, ms):
+def path_roofline(M, K, N, T, C, U, R, peaks, ms, entries=None):
     """The path roofline as the scope table's measurement rule states it:
     T_roof = max(2MKN / P_tc, B_alg / BW_hbm) with
     B_alg = 2KN + 4K*U + 2MK + 4MK + 2*M*(N/T)*(2+3C) + 4*R*N
@@ -291,7 +302,14 @@ def path_roofline(M, K, N, T, C, U, R, peaks, ms):
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = b_alg / (peaks["hbm_gbs"] * 1e9)
     t_roof = max(t_tc, t_hbm)
+    # Reported, not the target: the fp32 ALU time of the sparse products (one
+    # FMA per (entry, k) for each of the dot and the axpy: 4K FLOP per listed
+    # entry) against B200's fp32 FMA rate (148 SMs x 128 lanes x 2 FLOP at
+    # 1965 MHz = 74.4 TFLOP/s).
+    nnz = float(entries) if entries is not None else 0.0
+    t_alu = 4.0 * K * nnz / 74.4e12
     return {"t_roof_ms": t_roof * 1e3, "t_step_ms": ms, "frac": t_roof * 1e3 / ms,
+            "t_alu_sparse_ms": t_alu * 1e3,
             "bound": "tensor" if t_tc >= t_hbm else "hbm",
             "flops": flops, "bytes": b_alg, "P_tc_tflops": peaks["bf16_tflops"], "BW_hbm_gbs": peaks["hbm_gbs"],
             "U": U, "R": R, "bytes_fp32_vals_variant": b_build,
@@ -371,6 +389,20 @@ def measure_workload(tw, torch, dev, w, d, steps, warmup, flush, peaks, peak_kin
         ms = timed(step_read_status, check_words)
     n_launches = launches[0]
     ms_async = timed(step_async)
+
+    def timed_warm(fn):
+        # No flush between steps: whatever of the weights L2 keeps stays (secondary number).
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / steps
+
+    ms_warm = timed_warm(step_async)
     ms_sync = timed(step_sync_gate)
 
     # Per-kernel durations: the same steps again with an event pair around
@@ -403,6 +435,14 @@ def measure_workload(tw, torch, dev, w, d, steps, warmup, flush, peaks, peak_kin
         tw.dense_ffn(x, wg, wu, wd, h1, yd, bf16_h=True)
     dense_bf16h_ms = timed(lambda: tw.dense_ffn(x, wg, wu, wd, h1, yd, bf16_h=True))
     del h, h1, yd
+
+    # Sanity only: the same dense FFN with torch bf16 matmuls (cuBLAS) and
+    # elementwise kernels, h rounded to bf16.
+    def cublas_ffn():
+        return ((x @ wu.t()) * torch.relu(x @ wg.t())) @ wd
+    for _ in range(2):
+        cublas_ffn()
+    cublas_ms = timed(cublas_ffn)
 
     NT = N // T
     flops_gate = 2.0 * M * K * N
@@ -442,8 +482,12 @@ def measure_workload(tw, torch, dev, w, d, steps, warmup, flush, peaks, peak_kin
         "workload": w.name, "M": M, "K": K, "N": N, "T": T, "C": C, "R_cap": tb.R_cap,
         "ms_per_step": ms, "value": M / (ms * 1e-3),
         "ms_per_step_async": ms_async, "ms_per_step_sync_gate": ms_sync,
+        "ms_per_step_warm_l2": ms_warm,
+        "dense_cublas_sanity": {"ms_per_step": cublas_ms,
+                                "variant": "torch bf16 matmuls (cuBLAS) + elementwise, h in bf16; sanity only"},
         "sparsity": stats, "unique_units_gathered": U, "n_over": n_over,
-        "roofline": roofline, "path_roofline": path_roofline(M, K, N, T, C, U, n_over, peaks, ms),
+        "roofline": roofline,
+        "path_roofline": path_roofline(M, K, N, T, C, U, n_over, peaks, ms, entries=stats["twell_entries"]),
         "kernels": kernels,
         "dense": {"ms_per_step": dense_ms, "value": M / (dense_ms * 1e-3), "unit": UNIT,
                   "variant": "dense_ffn_fwd: h as bf16 hi + lo, held to the same y rule as the sparse path"},
@@ -724,8 +768,11 @@ def run_native(args, rank, world, local_rank):
     cpu = None
     if not args.no_cpu_baseline:
         rate, rows, sec, cores = cpu_oracle_rate(d, w, rows_target_s=12.0)
+        drate, drows, dsec = cpu_dense_oracle_rate(d, w)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
-               "sample": f"{rows} seeded rows of {w.M} ({sec:.1f} s): fp64 gate, TwELL pack, sparse y"}
+               "sample": f"{rows} seeded rows of {w.M} ({sec:.1f} s): fp64 gate, TwELL pack, sparse y",
+               "dense_oracle": {"value": drate, "unit": UNIT,
+                                "sample": f"{drows} seeded rows ({dsec:.1f} s): fp64 dense FFN, every hidden unit"}}
 
     value = job_throughput(world, w.M, ms)
     line = {
@@ -742,7 +789,9 @@ def run_native(args, rank, world, local_rank):
         "n_over": head["n_over"],
         "roofline": head["roofline"],
         "path_roofline": path_roofline(w.M, w.K, w.N, w.T, w.C, head["unique_units_gathered"], head["n_over"],
-                                       peaks, ms),
+                                       peaks, ms, entries=head["sparsity"]["twell_entries"]),
+        "ms_per_step_warm_l2": head["ms_per_step_warm_l2"],
+        "dense_cublas_sanity": head["dense_cublas_sanity"],
         "kernels": head["kernels"],
         "dense": head["dense"], "dense_bf16h": head["dense_bf16h"],
         "speedup_vs_dense": head["dense"]["ms_per_step"] / ms,
