@@ -22,10 +22,12 @@
 //                every entry stream through a per-warp ring; the warp adds
 //                du W_u^T + dz W_g^T into dx (vector atomics, dx cleared
 //                first) and appends (row, h, du, dz) to the unit's segment;
-//   4. units   : one warp per (unit, 256-column chunk) reads the unit's
-//                segment and the entries' x and dy chunks, and writes the
-//                chunk of the three weight-gradient rows (plain stores; units
-//                with no entry get zero rows).
+//   4. units   : one warp per (piece of up to 64 of a unit's entries,
+//                256-column chunk) reads the entries' x and dy chunks and
+//                writes the chunk of the three weight-gradient rows (plain
+//                stores for units of one piece, zero rows for units with no
+//                entry; vector atomics into rows the row pass cleared for
+//                units of several pieces).
 #pragma once
 
 #include "epilogues.cuh"
@@ -63,6 +65,8 @@ struct BwdParams {
   int gather_overflow; // 1: overflow tiles also go through the row pass (else the dense-row GEMMs)
   int* row_entries;    // [M] TwELL entries per row
   int* row_units;      // [M + 1] first row-pass unit of each row (exclusive prefix)
+  int* piece_off;      // [N + 1] first unit-pass piece of each hidden unit (exclusive prefix)
+  int* piece_unit;     // [N + cap / 64] hidden unit of each unit-pass piece
   int stages, list_cap;
   int* ctrl;           // ctrl[kCtrlNOver]: slots in use
 };
@@ -97,37 +101,61 @@ __global__ void __launch_bounds__(256) twell_bwd_count_kernel(const BwdParams p)
 // run of consecutive values, the CTA scans the 1024 sums, and each thread
 // writes its run's offsets; out[n] is the total.  mode 0: the values are
 // in[i]; mode 1: the row-pass units of row i, ceil(in[i] / kBwdUnitEntries).
-constexpr int kBwdUnitEntries = 32;  // row-pass unit: at most this many TwELL entries
+// With `pieces` given (mode 0 over the per-unit counts), the same pass also
+// scans the unit-pass pieces of hidden unit i, max(1, ceil(in[i] /
+// kBwdPieceEntries)), into pieces[], and writes i into owner[pieces[i] ..
+// pieces[i + 1]).
+constexpr int kBwdUnitEntries = 32;   // row-pass unit: at most this many TwELL entries
+constexpr int kBwdPieceEntries = 64;  // unit-pass piece: at most this many entries of one hidden unit
 
-__device__ __forceinline__ int bwd_scan_value(const int* in, int i, int mode) {
-  const int v = in[i];
-  return mode == 0 ? v : (v + kBwdUnitEntries - 1) / kBwdUnitEntries;
+__device__ __forceinline__ int bwd_pieces(int c) {
+  return c > kBwdPieceEntries ? (c + kBwdPieceEntries - 1) / kBwdPieceEntries : 1;
 }
 
 __global__ void __launch_bounds__(1024) twell_bwd_scan_kernel(const int* __restrict__ in, int* __restrict__ out, int n,
-                                                              int mode) {
-  __shared__ int part[1024];
+                                                              int mode, int* __restrict__ pieces,
+                                                              int* __restrict__ owner) {
+  __shared__ int part[2][1024];
   griddep_launch_dependents();
   griddep_wait();
+  const int t = threadIdx.x;
   const int per = (n + 1023) / 1024;
-  const int a = threadIdx.x * per;
+  const int a = t * per;
   const int b = a + per < n ? a + per : n;
-  int s = 0;
-  for (int i = a; i < b; ++i) s += bwd_scan_value(in, i, mode);
-  part[threadIdx.x] = s;
+  int s = 0, q = 0;
+  for (int i = a; i < b; ++i) {
+    const int v = in[i];
+    s += mode == 0 ? v : (v + kBwdUnitEntries - 1) / kBwdUnitEntries;
+    q += bwd_pieces(v);
+  }
+  part[0][t] = s;
+  part[1][t] = q;
   __syncthreads();
   for (int o = 1; o < 1024; o <<= 1) {
-    const int v = threadIdx.x >= o ? part[threadIdx.x - o] : 0;
+    const int v0 = t >= o ? part[0][t - o] : 0;
+    const int v1 = t >= o ? part[1][t - o] : 0;
     __syncthreads();
-    part[threadIdx.x] += v;
+    part[0][t] += v0;
+    part[1][t] += v1;
     __syncthreads();
   }
-  int run = part[threadIdx.x] - s;  // exclusive start of this thread's run
+  int run = part[0][t] - s;   // exclusive start of this thread's run
+  int prun = part[1][t] - q;  // and of its pieces
   for (int i = a; i < b; ++i) {
+    const int v = in[i];
     out[i] = run;
-    run += bwd_scan_value(in, i, mode);
+    run += mode == 0 ? v : (v + kBwdUnitEntries - 1) / kBwdUnitEntries;
+    if (pieces != nullptr) {
+      pieces[i] = prun;
+      const int w = bwd_pieces(v);
+      for (int j = 0; j < w; ++j) owner[prun + j] = i;
+      prun += w;
+    }
   }
-  if (threadIdx.x == 1023) out[n] = part[1023];
+  if (t == 1023) {
+    out[n] = part[0][1023];
+    if (pieces != nullptr) pieces[n] = part[1][1023];
+  }
 }
 
 // ---------------------------------------------------------------- 3. rows
@@ -269,6 +297,17 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
   lp.T = p.T;
   lp.C = p.C;
 
+  // The weight-gradient rows of hidden units whose entries the unit pass cuts
+  // into several pieces are added into with atomics there: clear them here.
+  for (int n = blockIdx.x * (blockDim.x >> 5) + warp; n < p.N; n += gridDim.x * (blockDim.x >> 5)) {
+    if (p.cnt[n] <= kBwdPieceEntries) continue;
+    for (int k = lane * 4; k < p.K; k += 128) {
+      const int64_t o = static_cast<int64_t>(n) * p.K + k;
+      *reinterpret_cast<float4*>(p.dwd + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(p.dwu_t + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(p.dwg_t + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   const int64_t n_twell = p.row_units[p.M];  // units over TwELL tiles (rows cut by entries)
   const int chunks = p.T / 32;
   const int n_over = p.gather_overflow ? min(ld_acquire(p.ctrl + kCtrlNOver), p.r_cap) : 0;
@@ -398,25 +437,30 @@ __global__ void __launch_bounds__(256) twell_bwd_slot_operands_kernel(const floa
 }
 
 // ---------------------------------------------------------------- 4. units
-// Warp item = (unit n, chunk c of 256 columns); lane l holds columns
-// c*256 + 8l .. +8 of the three gradient rows.
+// Warp item = (piece, chunk c of 256 columns); a piece is up to 64 entries of
+// one hidden unit n, and lane l holds columns c*256 + 8l .. +8 of the three
+// gradient rows.  A unit with one piece stores its rows; the pieces of a unit
+// with more entries add into rows the row pass cleared.
 __global__ void __launch_bounds__(256) twell_bwd_units_kernel(const BwdParams p) {
   griddep_launch_dependents();
   griddep_wait();
   const int lane = threadIdx.x & 31;
   const int chunks = (p.K + 255) / 256;
-  const int64_t items = static_cast<int64_t>(p.N) * chunks;
+  const int64_t items = static_cast<int64_t>(p.piece_off[p.N]) * chunks;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
        it += stride) {
-    const int n = static_cast<int>(it / chunks);
-    const int k0 = static_cast<int>(it - static_cast<int64_t>(n) * chunks) * 256 + lane * 8;
+    const int piece = static_cast<int>(it / chunks);
+    const int k0 = static_cast<int>(it - static_cast<int64_t>(piece) * chunks) * 256 + lane * 8;
+    const int n = p.piece_unit[piece];
+    const int r = piece - p.piece_off[n];
+    const bool split = p.piece_off[n + 1] - p.piece_off[n] > 1;
     const bool in = k0 < p.K;
     float ad[8], au[8], ag[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) ad[e] = au[e] = ag[e] = 0.f;
-    const int e0 = p.off[n];
-    const int e1 = p.off[n + 1];
+    const int e0 = p.off[n] + r * kBwdPieceEntries;
+    const int e1 = min(p.off[n + 1], e0 + kBwdPieceEntries);
     for (int b = e0; b < e1; b += 32) {
       // Lane j holds entry b + j; the warp then walks them in order.
       BwdEntry mine = {0, 0.f, 0.f, 0.f};
@@ -449,12 +493,21 @@ __global__ void __launch_bounds__(256) twell_bwd_units_kernel(const BwdParams p)
     }
     if (in) {
       const int64_t o = static_cast<int64_t>(n) * p.K + k0;
-      reinterpret_cast<float4*>(p.dwd + o)[0] = make_float4(ad[0], ad[1], ad[2], ad[3]);
-      reinterpret_cast<float4*>(p.dwd + o)[1] = make_float4(ad[4], ad[5], ad[6], ad[7]);
-      reinterpret_cast<float4*>(p.dwu_t + o)[0] = make_float4(au[0], au[1], au[2], au[3]);
-      reinterpret_cast<float4*>(p.dwu_t + o)[1] = make_float4(au[4], au[5], au[6], au[7]);
-      reinterpret_cast<float4*>(p.dwg_t + o)[0] = make_float4(ag[0], ag[1], ag[2], ag[3]);
-      reinterpret_cast<float4*>(p.dwg_t + o)[1] = make_float4(ag[4], ag[5], ag[6], ag[7]);
+      float4* dd = reinterpret_cast<float4*>(p.dwd + o);
+      float4* du4 = reinterpret_cast<float4*>(p.dwu_t + o);
+      float4* dg4 = reinterpret_cast<float4*>(p.dwg_t + o);
+      const float4 a0 = make_float4(ad[0], ad[1], ad[2], ad[3]), a1 = make_float4(ad[4], ad[5], ad[6], ad[7]);
+      const float4 u0 = make_float4(au[0], au[1], au[2], au[3]), u1 = make_float4(au[4], au[5], au[6], au[7]);
+      const float4 g0 = make_float4(ag[0], ag[1], ag[2], ag[3]), g1 = make_float4(ag[4], ag[5], ag[6], ag[7]);
+      if (split) {
+        atomicAdd(dd, a0); atomicAdd(dd + 1, a1);
+        atomicAdd(du4, u0); atomicAdd(du4 + 1, u1);
+        atomicAdd(dg4, g0); atomicAdd(dg4 + 1, g1);
+      } else {
+        dd[0] = a0; dd[1] = a1;
+        du4[0] = u0; du4[1] = u1;
+        dg4[0] = g0; dg4[1] = g1;
+      }
     }
   }
 }

@@ -321,7 +321,7 @@ constexpr int kBwdMaxK = 2560;      // the row pass keeps x, dy and dx pieces of
 constexpr int kBwdGatherSlots = 8;  // up to this many slotted rows go through the gather passes
 
 struct BwdLayout {
-  size_t cnt, fill, row_entries, off, row_units, entries;
+  size_t cnt, fill, row_entries, off, row_units, piece_off, piece_unit, entries;
   // dense-row slots (R_pad = R_cap rounded up to 64)
   size_t dy_cat, dy_hi, dy_lo, x_pad, u, du_rows, dz_rows, h_t, du_t, dz_t;
   size_t total;
@@ -340,6 +340,9 @@ BwdLayout bwd_layout(int M, int K, int N, int T, int C, int R_cap) {
   L.row_entries = o; o = align256(o + size_t(M) * 4);
   L.off = o; o = align256(o + size_t(N + 1) * 4);
   L.row_units = o; o = align256(o + size_t(M + 1) * 4);
+  L.piece_off = o; o = align256(o + size_t(N + 1) * 4);
+  // pieces = sum over units of max(1, ceil(cnt / 64)) <= N + cap / 64
+  L.piece_unit = o; o = align256(o + (size_t(N) + size_t(L.cap / 64) + 1) * 4);
   L.entries = o; o = align256(o + size_t(L.cap) * sizeof(BwdEntry));
   L.dy_cat = o; o = align256(o + rp * 2 * K * 2);
   L.dy_hi = o; o = align256(o + rp * K * 2);
@@ -865,6 +868,8 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   p.row_entries = reinterpret_cast<int*>(sb + L.row_entries);
   p.off = reinterpret_cast<int*>(sb + L.off);
   p.row_units = reinterpret_cast<int*>(sb + L.row_units);
+  p.piece_off = reinterpret_cast<int*>(sb + L.piece_off);
+  p.piece_unit = reinterpret_cast<int*>(sb + L.piece_unit);
   p.entries = reinterpret_cast<BwdEntry*>(sb + L.entries);
   p.slot_row = tw->slot_row;
   p.r_cap = tw->R_cap;
@@ -880,14 +885,17 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
                      stream, p));
   TW_CUDA(trace_end(stream, "bwd_count"));
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, static_cast<const int*>(p.cnt), p.off, N, 0));
+  TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, static_cast<const int*>(p.cnt), p.off, N, 0,
+                     p.piece_off, p.piece_unit));
   TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, static_cast<const int*>(p.row_entries), p.row_units,
-                     M, 1));
+                     M, 1, static_cast<int*>(nullptr), static_cast<int*>(nullptr)));
   TW_CUDA(trace_end(stream, "bwd_scan"));
   ++g_launches;  // the bracket holds two scans
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_bwd_rows(p, dev.sms, stream));
   TW_CUDA(trace_end(stream, "bwd_rows"));
+  // Items: (piece, 256-column chunk); at least one piece per hidden unit, and
+  // about entries / 64 more.  The grid covers the SMs; warps stride.
   const int64_t items = static_cast<int64_t>(N) * ((K + 255) / 256);
   const int64_t ugrid = (items + 7) / 8;
   TW_CUDA(trace_begin(stream));
