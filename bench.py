@@ -411,7 +411,7 @@ def measure_workload(tw, torch, dev, w, d, steps, warmup, flush, peaks, peak_kin
     traces = []
     for i in range(steps):
         flush.fill_(i & 0xFF)
-        tr = tw.KernelTrace(capacity=8)
+        tr = tw.KernelTrace(capacity=16)
         with tr:
             step_async()
         traces.append(tr)
@@ -615,7 +615,7 @@ def measure_backward(tw, torch, dev, w, d, steps, warmup, flush, peaks):
     per = {}
     for i in range(min(steps, 5)):
         flush.fill_(i & 0xFF)
-        tr = tw.KernelTrace(capacity=8)
+        tr = tw.KernelTrace(capacity=16)
         with tr:
             bwd()
         torch.cuda.synchronize()
