@@ -54,6 +54,7 @@ def _run(w, d, dev, R_cap=None, seed=0):
            "dwg_t": _check("dwg_t", dg, ref["dwg_t"], idle),
            "dwu_t": _check("dwu_t", du, ref["dwu_t"], idle),
            "dwd": _check("dwd", dd, ref["dwd"], idle)}
+    _run.last_unit_entries = mask[h["row_slot"] < 0].sum(axis=0)  # TwELL entries per hidden unit
     return out, int(mask.sum()), int((h["row_slot"] >= 0).sum())
 
 
@@ -77,3 +78,21 @@ def test_backward_workloads(name):
     w, d, dev = _workload(name)
     out, active, slotted = _run(w, d, dev, seed=3)
     print(name, out, active, slotted)
+
+
+@pytest.mark.parametrize("C,R_cap", [(32, None), (16, None), (12, 2000)])
+def test_backward_units_with_many_entries(C, R_cap):
+    # 5% activation over 2000 rows: about 100 TwELL entries per hidden unit, so
+    # the unit pass cuts units into pieces of at most 64 entries that add into
+    # the same weight-gradient rows.  C=32: no row overflows; C=16: a few rows
+    # do, and (at most 8 of them) their entries join the gather passes; C=12:
+    # dozens do, and go through the dense slot GEMMs.
+    w, d, dev = _small(2000, 192, 256, 128, C, None, seed=11, R_cap=R_cap)
+    out, active, slotted = _run(w, d, dev, R_cap=R_cap, seed=5)
+    per_unit = _run.last_unit_entries
+    assert per_unit.max() > 64, per_unit.max()
+    if C == 16:
+        assert 0 < slotted <= 8, slotted
+    if C == 12:
+        assert slotted > 8, slotted
+    print(C, out, active, slotted, int(per_unit.min()), int(per_unit.max()))
