@@ -182,12 +182,18 @@ twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint
  * with, per active (m, n): u = x_m W_u^T[n], dh = dy_m . W_d[n], h = u g,
  * du = dh g, dz = dh u (g = ReLU(z) from TwELL or the row's dense-row slot).
  * scratch: device, 256-byte aligned, >= twell_bwd_scratch_bytes(...) bytes
- * (per-unit counts and offsets, and a unit-major list of 16-byte entries
- * (row, h, du, dz): the hybrid activations transposed).  Limits: those of
- * twell_buf_init and K <= 2560.  Launches two memsets and four kernels
- * (count, scan, row pass, unit pass).  Asynchronous.  The sums over rows and
- * units are taken in an order that atomics decide, so repeated calls agree to
- * rounding, not bit for bit.
+ * (per-unit counts and offsets, the pieces of heavy units, a unit-major list
+ * of 16-byte entries (row, h, du, dz): the hybrid activations transposed, and
+ * the operands of the dense-slot GEMMs).  Limits: those of twell_buf_init and
+ * K <= 2560.
+ * Host side: the call first reads the number of slotted rows (one 4-byte
+ * device-to-host copy and a synchronize of `stream`), then queues the rest
+ * without waiting: two memsets (counters, dx) and five kernels (count, two
+ * scans, row pass, unit pass); with more than 8 slotted rows, also three
+ * memsets, an operand kernel and eight tensor-core GEMMs for those rows
+ * (with at most 8 their entries join the row and unit passes).  The sums
+ * over rows and units are taken in an order that atomics decide, so repeated
+ * calls agree to rounding, not bit for bit.
  */
 size_t twell_bwd_scratch_bytes(int M, int K, int N, int T, int C, int R_cap);
 twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
