@@ -146,9 +146,9 @@ twell_status twell_gate_pack(const uint16_t* x, const uint16_t* wg_t, int M, int
  * stream), then the dense-row path for overflow tiles (§3-6, §4-3).  wu_t, wd [N][K]
  * device bf16; y [M][K] device fp32, fully overwritten.  K must equal tw->K.
  * For M <= 256: y is cleared (a memset on `stream`) and one static-unit
- * kernel serves TwELL and overflow tiles (no dense-row GEMMs).  Asynchronous.  If the gate pass ran out of dense-row slots, the rows marked
- * -2 in row_slot miss their overflow tiles and twell_read_status returns
- * TWELL_ERR_CAPACITY.
+ * kernel serves TwELL and overflow tiles (no dense-row GEMMs).  Asynchronous.
+ * If the gate pass ran out of dense-row slots, the rows marked -2 in row_slot
+ * miss their overflow tiles and twell_read_status returns TWELL_ERR_CAPACITY.
  */
 twell_status twell_ffn_fwd(const uint16_t* x, const uint16_t* wu_t, const uint16_t* wd, const twell_buf* tw,
                            int K, float* y, cudaStream_t stream);
