@@ -17,8 +17,9 @@
 //                segment of a unit-major entry list (the hybrid transpose);
 //   3. rows    : static units: a row's TwELL entries cut into shares of at
 //                most 32 entries (by tile ranges, from a per-row count and
-//                a scan of the units per row), or, when only a few rows hold
-//                dense-row slots, one 32-column chunk of an overflow tile; the W_u^T, W_d and W_g^T rows of
+//                a scan of the units per row), or, when the slotted rows'
+//                entries go through the gather passes too, one 32-column
+//                chunk of an overflow tile; the W_u^T, W_d and W_g^T rows of
 //                every entry stream through a per-warp ring; the warp adds
 //                du W_u^T + dz W_g^T into dx (vector atomics, dx cleared
 //                first) and appends (row, h, du, dz) to the unit's segment;
@@ -56,13 +57,14 @@ struct BwdParams {
   float* dwg_t;
   float* dwu_t;
   float* dwd;
-  int* cnt;            // [N] entries per unit
+  int* cnt;            // [N] entries per unit (TwELL, then the overflow tiles' when gathered)
+  int* over_total;     // [1] active entries in the slotted rows' overflow tiles
   int* off;            // [N + 1] start of each unit's segment
   int* fill;           // [N] entries written so far per unit
   BwdEntry* entries;   // unit-major entry list
   const int* slot_row; // [R_cap] row of each dense-row slot
   int r_cap;
-  int gather_overflow; // 1: overflow tiles also go through the row pass (else the dense-row GEMMs)
+  int gather_overflow; // 1: overflow tiles also go through the row and unit passes (else the dense-row GEMMs)
   int* row_entries;    // [M] TwELL entries per row
   int* row_units;      // [M + 1] first row-pass unit of each row (exclusive prefix)
   int* piece_off;      // [N + 1] first unit-pass piece of each hidden unit (exclusive prefix)
@@ -72,28 +74,70 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------- 1. count
+// The positive gates of the slotted rows' overflow tiles, a warp per (slot,
+// tile) and a lane per column: each adds 1 to its unit's cnt (when cnt is
+// given).  Returns this lane's number of them.
+__device__ __forceinline__ int bwd_overflow_gates(const BwdParams& p, int* cnt) {
+  const int lane = threadIdx.x & 31;
+  const int NT = p.N / p.T;
+  const int n_over = min(ld_acquire(p.ctrl + kCtrlNOver), p.r_cap);
+  const int64_t items = static_cast<int64_t>(n_over) * NT;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  int found = 0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); i < items;
+       i += stride) {
+    const int slot = static_cast<int>(i / NT);
+    const int t = static_cast<int>(i - static_cast<int64_t>(slot) * NT);
+    const int row = p.slot_row[slot];
+    if (row < 0 || row >= p.M || p.counts[static_cast<int64_t>(row) * NT + t] <= p.C) continue;
+    const float4* g = reinterpret_cast<const float4*>(p.dense_rows + static_cast<int64_t>(slot) * p.N +
+                                                      static_cast<int64_t>(t) * p.T);
+    for (int j = lane; j < p.T / 4; j += 32) {
+      const float4 v = g[j];
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (e[i] > 0.f) {
+          ++found;
+          if (cnt != nullptr) atomicAdd(cnt + t * p.T + 4 * j + i, 1);
+        }
+      }
+    }
+  }
+  return found;
+}
+
 __global__ void __launch_bounds__(256) twell_bwd_count_kernel(const BwdParams p) {
   griddep_launch_dependents();
   griddep_wait();
   const int NT = p.N / p.T;
   const int64_t records = static_cast<int64_t>(p.M) * NT;
+  int over = 0;  // active entries of slotted rows' overflow tiles (their true counts)
   for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < records;
        r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int c = p.counts[r];
     if (c == 0) continue;
     const int m = static_cast<int>(r / NT);
-    const int t = static_cast<int>(r - static_cast<int64_t>(m) * NT);
-    if (c <= p.C) {
-      for (int s = 0; s < c; ++s) atomicAdd(p.cnt + t * p.T + p.idx[r * p.C + s], 1);
-      atomicAdd(p.row_entries + m, c);
-    } else if (p.gather_overflow) {
-      const int slot = p.row_slot[m];
-      if (slot < 0) continue;
-      const float* g = p.dense_rows + static_cast<int64_t>(slot) * p.N + static_cast<int64_t>(t) * p.T;
-      for (int j = 0; j < p.T; ++j)
-        if (g[j] > 0.f) atomicAdd(p.cnt + t * p.T + j, 1);
+    if (c > p.C) {
+      if (p.row_slot[m] >= 0) over += c;
+      continue;
     }
+    const int t = static_cast<int>(r - static_cast<int64_t>(m) * NT);
+    for (int s = 0; s < c; ++s) atomicAdd(p.cnt + t * p.T + p.idx[r * p.C + s], 1);
+    atomicAdd(p.row_entries + m, c);
   }
+  // The host picks the slotted rows' route from their number of entries.
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) over += __shfl_xor_sync(0xffffffffu, over, o);
+  if ((threadIdx.x & 31) == 0 && over > 0) atomicAdd(p.over_total, over);
+}
+
+// When the slotted rows go through the gather passes: their overflow entries
+// added to the units' counts.
+__global__ void __launch_bounds__(256) twell_bwd_overflow_units_kernel(const BwdParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  bwd_overflow_gates(p, p.cnt);
 }
 
 // ---------------------------------------------------------------- 2. scan
@@ -300,7 +344,7 @@ __global__ void __launch_bounds__(32 * bwd_max_warps<KV>(), 1) twell_bwd_rows_ke
   // The weight-gradient rows of hidden units whose entries the unit pass cuts
   // into several pieces are added into with atomics there: clear them here.
   for (int n = blockIdx.x * (blockDim.x >> 5) + warp; n < p.N; n += gridDim.x * (blockDim.x >> 5)) {
-    if (p.cnt[n] <= kBwdPieceEntries) continue;
+    if (p.off[n + 1] - p.off[n] <= kBwdPieceEntries) continue;
     for (int k = lane * 4; k < p.K; k += 128) {
       const int64_t o = static_cast<int64_t>(n) * p.K + k;
       *reinterpret_cast<float4*>(p.dwd + o) = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -32,6 +32,9 @@ thread_local int g_launches = 0;
 // the next fused-kernel launch on this thread, whose wait target is then made
 // unreachable; 0 = none.
 thread_local long long g_expire_wait_ns = 0;
+// Route of the slotted rows in twell_ffn_bwd on this thread
+// (twell_bwd_slot_route): 0 by cost, 1 the dense-slot GEMMs, 2 the gather passes.
+thread_local int g_bwd_slot_route = 0;
 
 // Optional launch tracing: events[2i] / events[2i+1] bracket the i-th kernel.
 struct Trace {
@@ -318,10 +321,24 @@ cudaError_t launch_fused_small(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
 
 // ---------------------------------------------------------------- backward
 constexpr int kBwdMaxK = 2560;      // the row pass keeps x, dy and dx pieces of a row in registers
-constexpr int kBwdGatherSlots = 8;  // up to this many slotted rows go through the gather passes
+constexpr int kBwdGatherSlots = 8;  // up to this many slotted rows always go through the gather passes
+
+// Whether the slotted rows' backward goes through the eight dense-slot GEMMs
+// rather than the gather passes, given R slotted rows holding `entries`
+// active entries.  Measured on one B200 (whole backward): the GEMMs cost
+// about 30 us + 26 ps per weight element N*K (launch- and tail-bound at these
+// row counts: M=2048 K=1536 N=4096 0.21 ms, M=8192 K=2048 N=5632 0.40 ms,
+// M=16384 K=2560 N=10240 0.70 ms), an entry in the gather passes about
+// 1.6 ps per K column.  The cut-over is taken a little short of the break-even
+// count, at 14 N + 12e6 / K entries.
+bool bwd_dense_slots(int R, long long entries, int N, int K) {
+  if (g_bwd_slot_route == 1) return R > 0;
+  if (g_bwd_slot_route == 2 || R <= kBwdGatherSlots) return false;
+  return entries > 14LL * N + 12000000LL / K;
+}
 
 struct BwdLayout {
-  size_t cnt, fill, row_entries, off, row_units, piece_off, piece_unit, entries;
+  size_t cnt, fill, row_entries, over_total, off, row_units, piece_off, piece_unit, entries;
   // dense-row slots (R_pad = R_cap rounded up to 64)
   size_t dy_cat, dy_hi, dy_lo, x_pad, u, du_rows, dz_rows, h_t, du_t, dz_t;
   size_t total;
@@ -338,6 +355,7 @@ BwdLayout bwd_layout(int M, int K, int N, int T, int C, int R_cap) {
   L.cnt = o; o = align256(o + size_t(N) * 4);
   L.fill = o; o = align256(o + size_t(N) * 4);
   L.row_entries = o; o = align256(o + size_t(M) * 4);
+  L.over_total = o; o = align256(o + 4);
   L.off = o; o = align256(o + size_t(N + 1) * 4);
   L.row_units = o; o = align256(o + size_t(M + 1) * 4);
   L.piece_off = o; o = align256(o + size_t(N + 1) * 4);
@@ -586,6 +604,12 @@ twell_status twell_test_expire_wait(long long limit_ns) {
   if (limit_ns != 0 && (limit_ns < 1000 || limit_ns > 1000000000))
     return fail(TWELL_ERR_INVALID, "limit_ns must be 0 or in [1000, 1000000000], got %lld", limit_ns);
   g_expire_wait_ns = limit_ns;
+  return TWELL_OK;
+}
+
+twell_status twell_bwd_slot_route(int route) {
+  if (route < 0 || route > 2) return fail(TWELL_ERR_INVALID, "route must be 0, 1 or 2, got %d", route);
+  g_bwd_slot_route = route;
   return TWELL_OK;
 }
 
@@ -848,15 +872,6 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   DeviceInfo dev;
   if ((st = device_info(dev)) != TWELL_OK) return st;
 
-  // The number of slotted rows sizes the dense-row GEMMs: read it once.
-  int n_over = 0;
-  TW_CUDA(cudaMemcpyAsync(&n_over, tw->ctrl + kCtrlNOver, sizeof n_over, cudaMemcpyDeviceToHost, stream));
-  TW_CUDA(cudaStreamSynchronize(stream));
-  const int R = n_over < tw->R_cap ? n_over : tw->R_cap;
-  // A handful of slotted rows is cheaper through the gather passes than
-  // through eight GEMM launches.
-  const bool dense_slots = R > kBwdGatherSlots;
-
   uint8_t* sb = static_cast<uint8_t*>(scratch);
   BwdParams p = {};
   p.x = x; p.wg_t = wg_t; p.wu_t = wu_t; p.wd = wd; p.dy = dy;
@@ -866,6 +881,7 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   p.cnt = reinterpret_cast<int*>(sb + L.cnt);
   p.fill = reinterpret_cast<int*>(sb + L.fill);
   p.row_entries = reinterpret_cast<int*>(sb + L.row_entries);
+  p.over_total = reinterpret_cast<int*>(sb + L.over_total);
   p.off = reinterpret_cast<int*>(sb + L.off);
   p.row_units = reinterpret_cast<int*>(sb + L.row_units);
   p.piece_off = reinterpret_cast<int*>(sb + L.piece_off);
@@ -873,10 +889,9 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   p.entries = reinterpret_cast<BwdEntry*>(sb + L.entries);
   p.slot_row = tw->slot_row;
   p.r_cap = tw->R_cap;
-  p.gather_overflow = dense_slots ? 0 : 1;
   p.ctrl = tw->ctrl;
 
-  TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // unit counts, fill, row entries
+  TW_CUDA(cudaMemsetAsync(sb, 0, L.off, stream));  // unit counts, fill, row entries, overflow total
   TW_CUDA(cudaMemsetAsync(dx, 0, static_cast<size_t>(M) * K * sizeof(float), stream));
   const int64_t records = static_cast<int64_t>(M) * (N / tw->T);
   const int64_t cgrid = (records + 255) / 256;
@@ -884,6 +899,22 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   TW_CUDA(launch_pdl(twell_bwd_count_kernel, static_cast<int>(cgrid < 4 * dev.sms ? cgrid : 4 * dev.sms), 256, 0,
                      stream, p));
   TW_CUDA(trace_end(stream, "bwd_count"));
+  // The number of slotted rows and of their overflow entries choose the
+  // slotted rows' route: read both once.
+  int n_over = 0, n_over_entries = 0;
+  TW_CUDA(cudaMemcpyAsync(&n_over, tw->ctrl + kCtrlNOver, sizeof n_over, cudaMemcpyDeviceToHost, stream));
+  TW_CUDA(cudaMemcpyAsync(&n_over_entries, p.over_total, sizeof n_over_entries, cudaMemcpyDeviceToHost, stream));
+  TW_CUDA(cudaStreamSynchronize(stream));
+  const int R = n_over < tw->R_cap ? n_over : tw->R_cap;
+  const bool dense_slots = bwd_dense_slots(R, n_over_entries, N, K);
+  p.gather_overflow = dense_slots ? 0 : 1;
+  if (!dense_slots && n_over_entries > 0) {
+    TW_CUDA(trace_begin(stream));
+    TW_CUDA(launch_pdl(twell_bwd_overflow_units_kernel, static_cast<int>(cgrid < 4 * dev.sms ? cgrid : 4 * dev.sms),
+                       256, 0, stream, p));
+    TW_CUDA(trace_end(stream, "bwd_overflow_units"));
+  }
+
   TW_CUDA(trace_begin(stream));
   TW_CUDA(launch_pdl(twell_bwd_scan_kernel, 1, 1024, 0, stream, static_cast<const int*>(p.cnt), p.off, N, 0,
                      p.piece_off, p.piece_unit));

@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         "twell_ffn_fused": (I, [P, P, P, P, I, I, I, BP, P, IP, P]),
         "twell_bwd_scratch_bytes": (S, [I, I, I, I, I, I]),
         "twell_ffn_bwd": (I, [P, P, P, P, BP, P, I, P, P, P, P, P, S, P]),
+        "twell_bwd_slot_route": (I, [I]),
         "twell_read_status": (I, [BP, IP, IP, P]),
         "dense_ffn_fwd": (I, [P, P, P, P, I, I, I, P, P, P]),
         "dense_ffn_fwd_bf16h": (I, [P, P, P, P, I, I, I, P, P, P]),
@@ -345,6 +346,13 @@ def dense_ffn_noalloc(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, w
                                      y.data_ptr(), _stream(stream))
     _check(st, "dense_ffn_fwd_noalloc")
     return y
+
+
+def bwd_slot_route(route: int) -> None:
+    """twell_bwd_slot_route: 0 chooses the slotted rows' backward route by
+    their entry count, 1 forces the dense-slot GEMMs, 2 the gather passes
+    (for the calling thread)."""
+    _check(lib().twell_bwd_slot_route(int(route)), "twell_bwd_slot_route")
 
 
 def test_expire_wait(limit_ns: int) -> None:

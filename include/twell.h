@@ -186,16 +186,31 @@ twell_status twell_ffn_fused(const uint16_t* x, const uint16_t* wg_t, const uint
  * of 16-byte entries (row, h, du, dz): the hybrid activations transposed, and
  * the operands of the dense-slot GEMMs).  Limits: those of twell_buf_init and
  * K <= 2560.
- * Host side: the call first reads the number of slotted rows (one 4-byte
- * device-to-host copy and a synchronize of `stream`), then queues the rest
- * without waiting: two memsets (counters, dx) and five kernels (count, two
- * scans, row pass, unit pass); with more than 8 slotted rows, also three
- * memsets, an operand kernel and eight tensor-core GEMMs for those rows
- * (with at most 8 their entries join the row and unit passes).  The sums
- * over rows and units are taken in an order that atomics decide, so repeated
- * calls agree to rounding, not bit for bit.
+ * Host side: the call queues two memsets (counters, dx) and the count
+ * kernel, which also counts the active entries of the slotted rows' overflow
+ * tiles; it reads that count and the number of slotted rows R (two 4-byte
+ * device-to-host copies and a synchronize of `stream`), then queues the rest
+ * without waiting: four kernels (two scans, row pass, unit pass), and before
+ * them, when the slotted rows go through the gather passes, one kernel that
+ * adds their entries to the per-unit counts.  The
+ * slotted rows take one of two routes (twell_bwd_slot_route):
+ * their entries join the row and unit passes, or three memsets, an operand
+ * kernel and eight tensor-core GEMMs cover them.  By default the GEMMs are
+ * taken when R > 8 and the rows hold more than 14 N + 12e6 / K entries (the
+ * measured break-even on one B200, a little short of it).  The sums over rows
+ * and units are taken in an order that atomics decide, so repeated calls
+ * agree to rounding, not bit for bit.
  */
 size_t twell_bwd_scratch_bytes(int M, int K, int N, int T, int C, int R_cap);
+
+/*
+ * Route of the slotted rows in the following twell_ffn_bwd calls on the
+ * calling thread: 0 by the entry count above (the default), 1 always the
+ * dense-slot GEMMs (when any row is slotted), 2 always the gather passes.
+ * Both routes compute the same gradients (to rounding).  Returns
+ * TWELL_ERR_INVALID for any other value.
+ */
+twell_status twell_bwd_slot_route(int route);
 twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16_t* wu_t, const uint16_t* wd,
                            const twell_buf* tw, const float* dy, int K, float* dx, float* dwg_t, float* dwu_t,
                            float* dwd, void* scratch, size_t scratch_bytes, cudaStream_t stream);

@@ -117,6 +117,14 @@ def test_expire_wait_hook_validates_its_limit():
     assert L.twell_test_expire_wait(0) == tw.OK       # disarm: nothing launched here
 
 
+def test_bwd_slot_route_validates_its_value():
+    L = tw.lib()
+    for bad in (-1, 3):
+        assert L.twell_bwd_slot_route(bad) == tw.ERR_INVALID
+    for ok in (1, 2, 0):  # ends on the default
+        assert L.twell_bwd_slot_route(ok) == tw.OK
+
+
 def test_noalloc_rejects_oversize_before_any_cuda_call():
     L = tw.lib()
     p = 1 << 33

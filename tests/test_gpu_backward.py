@@ -40,12 +40,16 @@ def _check(name, got, ref, zero_rows=None):
     return err / rms
 
 
-def _run(w, d, dev, R_cap=None, seed=0):
+def _run(w, d, dev, R_cap=None, seed=0, route=0):
     t = tw.TwellBuffers(w.M, w.K, w.N, w.T, w.C, R_cap=R_cap if R_cap is not None else w.R_cap)
     tw.gate_pack(dev["x"], dev["wg_t"], t, sync=True)
     dy = np.random.default_rng(seed).standard_normal((w.M, w.K)).astype(np.float32)
-    dx, dg, du, dd = tw.ffn_bwd(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"], t, torch.from_numpy(dy).cuda())
-    torch.cuda.synchronize()
+    tw.bwd_slot_route(route)
+    try:
+        dx, dg, du, dd = tw.ffn_bwd(dev["x"], dev["wg_t"], dev["wu_t"], dev["wd"], t, torch.from_numpy(dy).cuda())
+        torch.cuda.synchronize()
+    finally:
+        tw.bwd_slot_route(0)
     h = t.to_host()
     mask = _active_mask(h, w.N, w.T, w.C)
     ref = ob.ffn_backward(d["x"], d["wg_t"], d["wu_t"], d["wd"], dy.astype(np.float64), active=mask)
@@ -65,9 +69,10 @@ def test_backward_small_shapes(M, T, C):
     print(M, T, C, out, active, slotted)
 
 
-def test_backward_all_gates_on_goes_through_the_dense_rows():
+@pytest.mark.parametrize("route", [0, 1, 2])
+def test_backward_all_gates_on_goes_through_the_dense_rows(route):
     w, d, dev = _small(40, 128, 512, 128, 4, bias=-1e2, seed=2, R_cap=40)
-    out, active, slotted = _run(w, d, dev, R_cap=40)
+    out, active, slotted = _run(w, d, dev, R_cap=40, route=route)
     assert slotted == 40 and active == 40 * 512
     print(out)
 
@@ -80,15 +85,25 @@ def test_backward_workloads(name):
     print(name, out, active, slotted)
 
 
-@pytest.mark.parametrize("C,R_cap", [(32, None), (16, None), (12, 2000)])
-def test_backward_units_with_many_entries(C, R_cap):
+@pytest.mark.parametrize("route", [1, 2])
+def test_backward_slotted_rows_by_either_route(route):
+    # 201 of 2048 rows hold dense-row slots (half of all active entries):
+    # the dense-slot GEMMs and the gather passes both meet the rule.
+    w, d, dev = _workload("m2048_k1536_n4096_p99_lognormal05")
+    out, active, slotted = _run(w, d, dev, seed=3, route=route)
+    assert slotted > 8
+    print(route, out, active, slotted)
+
+
+@pytest.mark.parametrize("C,R_cap,route", [(32, None, 0), (16, None, 0), (12, 2000, 0), (12, 2000, 1)])
+def test_backward_units_with_many_entries(C, R_cap, route):
     # 5% activation over 2000 rows: about 100 TwELL entries per hidden unit, so
     # the unit pass cuts units into pieces of at most 64 entries that add into
     # the same weight-gradient rows.  C=32: no row overflows; C=16: a few rows
     # do, and (at most 8 of them) their entries join the gather passes; C=12:
-    # dozens do, and go through the dense slot GEMMs.
+    # dozens do, through either route.
     w, d, dev = _small(2000, 192, 256, 128, C, None, seed=11, R_cap=R_cap)
-    out, active, slotted = _run(w, d, dev, R_cap=R_cap, seed=5)
+    out, active, slotted = _run(w, d, dev, R_cap=R_cap, seed=5, route=route)
     per_unit = _run.last_unit_entries
     assert per_unit.max() > 64, per_unit.max()
     if C == 16:
