@@ -629,6 +629,9 @@ def measure_backward(tw, torch, dev, w, d, steps, warmup, flush, peaks):
     return {"workload": w.name, "M": M, "K": K, "N": N, "ms": ms, "tokens_per_s": M / (ms * 1e-3),
             "n_over": n_over, "twell_entries": stats["twell_entries"], "status": st,
             "kernels_ms": {k: sum(v) / len(v) for k, v in per.items()},
+            # which route the library chose for the slotted rows (seen in the trace)
+            "slotted_rows_route": "dense-slot GEMMs" if any(k.startswith("bwd_slot_") for k in per)
+                                  else "gather passes",
             "torch_dense_backward_ms": dense_ms,
             "torch_dense_backward": "bf16 torch matmuls (cuBLAS) and elementwise ops, recomputing z and u; "
                                     "context only, not held to the y rule",
