@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(256) twell_bwd_overflow_units_kernel(const Bwd
 // pieces[i + 1]).
 constexpr int kBwdUnitEntries = 32;   // row-pass unit: at most this many TwELL entries
 constexpr int kBwdPieceEntries = 64;  // unit-pass piece: at most this many entries of one hidden unit
+constexpr int kBwdUnitBatch = 2;      // unit pass: entries whose loads are in flight together
 
 __device__ __forceinline__ int bwd_pieces(int c) {
   return c > kBwdPieceEntries ? (c + kBwdPieceEntries - 1) / kBwdPieceEntries : 1;
@@ -510,28 +511,51 @@ __global__ void __launch_bounds__(256) twell_bwd_units_kernel(const BwdParams p)
       BwdEntry mine = {0, 0.f, 0.f, 0.f};
       if (b + lane < e1) mine = p.entries[b + lane];
       const int cntb = e1 - b < 32 ? e1 - b : 32;
-      for (int j = 0; j < cntb; ++j) {
-        const int m = __shfl_sync(0xffffffffu, mine.m, j);
-        const float h = __shfl_sync(0xffffffffu, mine.h, j);
-        const float du = __shfl_sync(0xffffffffu, mine.du, j);
-        const float dz = __shfl_sync(0xffffffffu, mine.dz, j);
-        if (in) {
-          const uint4 xq = *reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.K + k0);
-          const float4 d0 = *reinterpret_cast<const float4*>(p.dy + static_cast<int64_t>(m) * p.K + k0);
-          const float4 d1 = *reinterpret_cast<const float4*>(p.dy + static_cast<int64_t>(m) * p.K + k0 + 4);
-          const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-          const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+      // kBwdUnitBatch entries per step, their x and dy loads issued before any is
+      // used.  Past the last entry a step loads the row of lane (j & 31)'s
+      // entry (row 0 for lanes past e1) and skips its arithmetic.
+      for (int j0 = 0; j0 < cntb; j0 += kBwdUnitBatch) {
+        int m[kBwdUnitBatch];
+        float h[kBwdUnitBatch], du[kBwdUnitBatch], dz[kBwdUnitBatch];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float xlo = __uint_as_float(xw[e] << 16);
-            const float xhi = __uint_as_float(xw[e] & 0xFFFF0000u);
-            au[2 * e] = fmaf(du, xlo, au[2 * e]);
-            au[2 * e + 1] = fmaf(du, xhi, au[2 * e + 1]);
-            ag[2 * e] = fmaf(dz, xlo, ag[2 * e]);
-            ag[2 * e + 1] = fmaf(dz, xhi, ag[2 * e + 1]);
+        for (int q = 0; q < kBwdUnitBatch; ++q) {
+          const int j = (j0 + q) & 31;
+          const bool ok = j0 + q < cntb;
+          m[q] = __shfl_sync(0xffffffffu, mine.m, j);
+          const float hq = __shfl_sync(0xffffffffu, mine.h, j);
+          const float uq = __shfl_sync(0xffffffffu, mine.du, j);
+          const float zq = __shfl_sync(0xffffffffu, mine.dz, j);
+          h[q] = ok ? hq : 0.f;
+          du[q] = ok ? uq : 0.f;
+          dz[q] = ok ? zq : 0.f;
+        }
+        if (in) {
+          uint4 xq[kBwdUnitBatch];
+          float4 d0[kBwdUnitBatch], d1[kBwdUnitBatch];
+#pragma unroll
+          for (int q = 0; q < kBwdUnitBatch; ++q) {
+            const int64_t row = static_cast<int64_t>(m[q]) * p.K + k0;
+            xq[q] = *reinterpret_cast<const uint4*>(p.x + row);
+            d0[q] = *reinterpret_cast<const float4*>(p.dy + row);
+            d1[q] = *reinterpret_cast<const float4*>(p.dy + row + 4);
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ad[e] = fmaf(h, dv[e], ad[e]);
+          for (int q = 0; q < kBwdUnitBatch; ++q) {
+            if (j0 + q >= cntb) break;  // the same for the whole warp
+            const float dv[8] = {d0[q].x, d0[q].y, d0[q].z, d0[q].w, d1[q].x, d1[q].y, d1[q].z, d1[q].w};
+            const uint32_t xw[4] = {xq[q].x, xq[q].y, xq[q].z, xq[q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float xlo = __uint_as_float(xw[e] << 16);
+              const float xhi = __uint_as_float(xw[e] & 0xFFFF0000u);
+              au[2 * e] = fmaf(du[q], xlo, au[2 * e]);
+              au[2 * e + 1] = fmaf(du[q], xhi, au[2 * e + 1]);
+              ag[2 * e] = fmaf(dz[q], xlo, ag[2 * e]);
+              ag[2 * e + 1] = fmaf(dz[q], xhi, ag[2 * e + 1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ad[e] = fmaf(h[q], dv[e], ad[e]);
+          }
         }
       }
     }
