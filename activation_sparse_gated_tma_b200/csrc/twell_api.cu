@@ -929,9 +929,14 @@ twell_status twell_ffn_bwd(const uint16_t* x, const uint16_t* wg_t, const uint16
   // about entries / 64 more.  The grid covers the SMs; warps stride.
   const int64_t items = static_cast<int64_t>(N) * ((K + 255) / 256);
   const int64_t ugrid = (items + 7) / 8;
+  // A plain launch: launched early (programmatic serialisation) the unit
+  // pass's CTAs are placed while the row pass runs, and the whole backward was
+  // slower (M=16384 K=2560 N=10240: 2.93 ms against 2.66 ms; M=8192 K=2048
+  // N=5632: 1.20 against 1.19 ms).  griddepcontrol.wait in the kernel is then
+  // a no-op.
   TW_CUDA(trace_begin(stream));
-  TW_CUDA(launch_pdl(twell_bwd_units_kernel, static_cast<int>(ugrid < 8 * dev.sms ? ugrid : 8 * dev.sms), 256, 0,
-                     stream, p));
+  twell_bwd_units_kernel<<<static_cast<int>(ugrid < 8 * dev.sms ? ugrid : 8 * dev.sms), 256, 0, stream>>>(p);
+  TW_CUDA(cudaGetLastError());
   TW_CUDA(trace_end(stream, "bwd_units"));
   if (!dense_slots) return TWELL_OK;
 
